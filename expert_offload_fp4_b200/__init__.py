@@ -1,0 +1,9 @@
+"""B200 (sm_100a) hot path of one FreeToken-style MoE layer with FP4 experts
+offloaded to pinned host memory: router, LRU expert-slot pool in HBM, copy-engine
+miss streaming, FP4 SwiGLU expert FFN, router-weighted combine, and the q*
+bandwidth split.  The work is in libmoe_fp4.so (include/moe_fp4.h); this package
+is its Python binding."""
+from . import _lib  # noqa: F401
+from .api import (Lookup, Pool, combine, dequant_slot, expert_ffn, qstar_split,  # noqa: F401
+                  route, route_workspace_bytes, set_wait_limits, slot_lookup, stream_misses)
+from .layer import DecodeLayer  # noqa: F401

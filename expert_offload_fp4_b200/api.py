@@ -1,0 +1,169 @@
+"""Thin Python binding of libmoe_fp4.so: argument marshalling only.
+
+Device buffers are torch tensors (their data_ptr is passed); streams are
+torch.cuda.Stream objects (their cuda_stream handle is passed).  Every step of
+the MoE layer runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+import torch
+
+from . import _lib as L
+
+FMT = {"mxfp4": L.MOE_MXFP4, "nvfp4": L.MOE_NVFP4}
+
+
+def _p(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _np(a, dt):
+    a = np.ascontiguousarray(a, dtype=dt)
+    return a, a.ctypes.data_as(C.c_void_p)
+
+
+class Pool:
+    """The library-owned expert store: pinned host blocks, HBM slots, LRU state."""
+
+    def __init__(self, H, I, E, k, L_layers, fmt, n_slots, max_tokens=8, host_layers=0):
+        self.lib = L.load()
+        self.cfg = L.MoeConfig(H, I, E, k, L_layers, FMT[fmt], n_slots, max_tokens, host_layers)
+        self.H, self.I, self.E, self.k, self.L = H, I, E, k, L_layers
+        self.fmt, self.n_slots, self.max_tokens = fmt, n_slots, max_tokens
+        self.host_layers = host_layers or L_layers
+        h = C.c_void_p()
+        L.check("moe_pool_create", self.lib.moe_pool_create(C.byref(self.cfg), C.byref(h)))
+        self.handle = h
+        self.block_bytes = self.lib.moe_expert_block_bytes(C.byref(self.cfg))
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self.lib.moe_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def load_expert(self, layer, expert, tensors):
+        """tensors: {"gate"|"up"|"down": (codes uint8, scales uint8, tensor_scale)}"""
+        src = L.ExpertSrc()
+        keep = []
+        for i, name in enumerate(("gate", "up", "down")):
+            c, s, ts = tensors[name]
+            c, cp = _np(c, np.uint8)
+            s, sp = _np(s, np.uint8)
+            keep += [c, s]
+            src.codes_h[i] = cp.value
+            src.scales_h[i] = sp.value
+            src.tensor_scale[i] = float(ts)
+        L.check("moe_pool_load_expert",
+                self.lib.moe_pool_load_expert(self.handle, int(layer), int(expert), C.byref(src)))
+
+    def read_state(self):
+        sk = np.empty(self.n_slots, np.int32)
+        sc = np.empty(self.n_slots, np.uint64)
+        ks = np.empty(self.L * self.E, np.int32)
+        g = np.zeros(1, np.uint64)
+        L.check("moe_pool_read_state", self.lib.moe_pool_read_state(
+            self.handle, sk.ctypes.data_as(C.c_void_p), sc.ctypes.data_as(C.c_void_p),
+            ks.ctypes.data_as(C.c_void_p), g.ctypes.data_as(C.c_void_p)))
+        return dict(slot_key=sk, slot_clock=sc, key_slot=ks, clock=int(g[0]))
+
+    def stats(self):
+        st = L.Stats()
+        L.check("moe_pool_stats", self.lib.moe_pool_stats(self.handle, C.byref(st)))
+        return {f: getattr(st, f) for f, _ in L.Stats._fields_}
+
+    def slot_ptr(self, slot):
+        p, n = C.c_void_p(), C.c_size_t()
+        L.check("moe_pool_slot_ptr", self.lib.moe_pool_slot_ptr(self.handle, int(slot), C.byref(p), C.byref(n)))
+        return p.value, n.value
+
+
+def route_workspace_bytes(T, E):
+    return L.load().moe_route_workspace_bytes(int(T), int(E))
+
+
+def route(x, wr, bias, k, renormalize, idx, w, workspace, stream=None):
+    T, H = x.shape
+    E = wr.shape[0]
+    L.check("moe_route", L.load().moe_route(
+        _p(x), _p(wr), _p(bias), T, H, E, int(k), int(renormalize), _p(idx), _p(w),
+        _p(workspace), workspace.numel() * workspace.element_size(), _s(stream)))
+
+
+class Lookup:
+    """Host-side result of one slot lookup (arrays sized for the call)."""
+
+    def __init__(self, cap):
+        self.uniq = np.zeros(cap, np.int32)
+        self.is_hit = np.zeros(cap, np.int32)
+        self.misses = (L.Miss * cap)()
+        self.res = L.LookupResult(0, 0, self.uniq.ctypes.data_as(C.POINTER(C.c_int32)),
+                                  self.is_hit.ctypes.data_as(C.POINTER(C.c_int32)), self.misses)
+
+    @property
+    def n_uniq(self):
+        return self.res.n_uniq
+
+    @property
+    def n_miss(self):
+        return self.res.n_miss
+
+    def miss_list(self):
+        return [(m.expert, m.slot, m.ticket, m.evicted_key) for m in self.misses[:self.res.n_miss]]
+
+
+def slot_lookup(pool, layer, idx, slot_of, result=None, stream=None):
+    T, k = idx.shape
+    if result is None:
+        result = Lookup(min(T * k, pool.E))
+    L.check("moe_slot_lookup", pool.lib.moe_slot_lookup(
+        pool.handle, int(layer), _p(idx), T, k, _p(slot_of), C.byref(result.res), _s(stream)))
+    return result
+
+
+def stream_misses(pool, layer, lookup, copy_stream):
+    L.check("moe_stream_misses", pool.lib.moe_stream_misses(
+        pool.handle, int(layer), lookup.misses, lookup.res.n_miss, _s(copy_stream)))
+
+
+def expert_ffn(pool, layer, x, idx, w, slot_of, y_part, status, stream=None):
+    T = x.shape[0]
+    L.check("moe_expert_ffn", pool.lib.moe_expert_ffn(
+        pool.handle, int(layer), _p(x), T, _p(idx), _p(w), _p(slot_of), _p(y_part), _p(status),
+        _s(stream)))
+
+
+def combine(y_part, y, stream=None):
+    T, k, H = y_part.shape
+    L.check("moe_combine", L.load().moe_combine(_p(y_part), T, k, H, _p(y), _s(stream)))
+
+
+def qstar_split(m, b_pcie, b_host):
+    qg, qc, r = C.c_int(), C.c_int(), C.c_double()
+    L.check("qstar_split", L.load().qstar_split(int(m), float(b_pcie), float(b_host),
+                                                C.byref(qg), C.byref(qc), C.byref(r)))
+    return qg.value, qc.value, r.value
+
+
+def dequant_slot(pool, slot, key, which, out, stream=None):
+    L.check("moe_dequant_slot", pool.lib.moe_dequant_slot(
+        pool.handle, int(slot), int(key), int(which), _p(out), _s(stream)))
+
+
+def set_wait_limits(ready_ms, dep_ms, pipe_ms):
+    L.check("moe_set_wait_limits", L.load().moe_set_wait_limits(float(ready_ms), float(dep_ms),
+                                                                 float(pipe_ms)))

@@ -1,0 +1,171 @@
+// Internal declarations shared by the library's translation units: the pool
+// object, error reporting, and thin wrappers over sm_100a PTX (mbarrier,
+// bulk asynchronous copies, bounded waits on the global timer).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <stdint.h>
+#include <string>
+
+#include "../../include/moe_fp4.h"
+
+namespace moe {
+
+// ----------------------------------------------------------------- errors
+
+void set_error(const std::string& msg);
+int fail(int code, const std::string& msg);
+int cuda_fail(cudaError_t e, const char* what);
+
+#define MOE_CUDA_TRY(expr)                                   \
+    do {                                                     \
+        cudaError_t e_ = (expr);                             \
+        if (e_ != cudaSuccess) return cuda_fail(e_, #expr);  \
+    } while (0)
+
+// ----------------------------------------------------------------- limits
+
+constexpr int kMaxE = 1024;          // experts per layer
+constexpr int kMaxK = 32;            // experts per token
+constexpr int kMaxDecodeT = 16;      // tokens of one decode FFN call
+constexpr int kMaxDecodePairs = 128; // (token, rank) pairs of one decode FFN call
+constexpr int kMaxSlots = 1 << 20;
+
+// Per-call output of the lookup kernel, in mapped pinned host memory.
+struct LookupOut {
+    int n_uniq, n_miss, status, seq;
+    int32_t uniq[kMaxE];
+    int32_t is_hit[kMaxE];
+    moe_miss miss[kMaxE];
+};
+
+// Byte layout of one expert block (4096-aligned tensors).
+struct BlockLayout {
+    size_t off[6];     // gate codes, gate scales, up codes, up scales, down codes, down scales
+    size_t bytes;      // whole block, multiple of 4096
+};
+
+BlockLayout block_layout(const moe_config& c);
+
+}  // namespace moe
+
+struct moe_pool {
+    moe_config cfg;
+    int bs;                       // elements per block scale
+    moe::BlockLayout lay;
+    int host_layers;
+    int device;
+    int num_sms;
+    // storage
+    uint8_t* slots;               // device [n_slots][block]
+    uint8_t* host;                // pinned [host_layers][E][block]
+    uint8_t* host_loaded;         // host flags [host_layers * E]
+    // LRU metadata (device)
+    int32_t* slot_key;            // [n_slots]
+    unsigned long long* slot_clock;  // [n_slots]
+    int32_t* key_slot;            // [L*E]
+    unsigned long long* clock;    // [1]
+    uint32_t* ticket;             // [1]
+    uint32_t* need;               // [n_slots] ticket the slot must show before use
+    uint32_t* ready;              // [n_slots] ticket published by the copy stream
+    float* tscale;                // [L*E*3] NVFP4 tensor scales
+    // lookup output
+    moe::LookupOut* lk_h;         // mapped pinned
+    moe::LookupOut* lk_d;         // its device alias
+    cudaEvent_t lk_event;
+    // decode FFN scratch
+    float* hbuf;                  // [kMaxDecodePairs][I] fp32
+    unsigned int* hamax;          // [kMaxDecodePairs] |h| max as float bits
+    unsigned int* ctr;            // [kMaxDecodePairs] h rows done per group, then done + abort
+    // copy engine ready-flag write
+    void* write_value32;          // cuStreamWriteValue32 entry point
+    moe_stats stats;
+};
+
+// ----------------------------------------------------------------- PTX wrappers
+#ifdef __CUDACC__
+namespace moe {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;"
+        " selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase; false after `limit_ns` of global time.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    unsigned long long t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > limit_ns) return false;
+    }
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_sys_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Named barrier over `nthreads` threads (a multiple of 32) with id `id` (1..15).
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+}  // namespace moe
+#endif

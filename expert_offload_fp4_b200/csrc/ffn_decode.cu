@@ -1,0 +1,683 @@
+// K4 decode expert FFN, K5 combine, and the slot dequantiser.
+//
+// K4 is one persistent kernel over the unique experts ("groups") of a decode
+// call.  Work items, in a fixed order that every CTA derives alike:
+//   A(g, rb): RA rows of gate and the same RA rows of up of group g -> h rows
+//   B(g, rb): RB rows of down of group g -> weighted outputs y_part
+// all A items first, then all B items; CTA c takes items c, c + grid, ...
+// Groups are ordered by the ticket their slot must show, so resident experts
+// come first and missed ones in the order the copy engine delivers them.
+//
+// Warp specialisation: warp NC (the producer) streams each item's FP4 codes and
+// block scales with 1-D TMA bulk copies into a ring of shared-memory stages
+// (mbarrier full/empty pairs); for a missed expert it first waits (bounded) for
+// the slot's ready flag written by the copy stream.  Warps 0..NC-1 (consumers)
+// decode E2M1 pairs with cvt.rn.f16x2.e2m1x2 and accumulate with the mixed
+// fma.rn.f32.f16 (exact products, fp32 sums) against activations held in f16
+// after a per-token power-of-two scale (bf16 x is exact in f16 that way; h is
+// rounded to f16's 11 significant bits).  A block's partial sum is scaled by
+// its E8M0 / E4M3 scale in fp32; the NVFP4 tensor scale and the activation
+// scale are applied per row.  A items publish h rows and bump a per-group
+// counter; B items wait (bounded) until all I rows of h exist.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kNC = 8;                       // consumer warps
+constexpr int kFfnThreads = (kNC + 1) * 32;  // + one producer warp
+constexpr int kAbortIdx = kMaxDecodePairs;   // ctr[kAbortIdx] = abort flag
+constexpr int kDoneIdx = kMaxDecodePairs + 1;
+
+struct Group {
+    int expert, slot, M, pos;
+    float ts[3];
+    uint8_t tok[kMaxDecodeT];
+    uint8_t rank[kMaxDecodeT];
+};
+
+struct FfnArgs {
+    const uint16_t* x;
+    const int32_t* idx;
+    const float* w;
+    const int32_t* slot_of;
+    float* y_part;
+    int* status;
+    const uint8_t* slots;
+    unsigned long long block_bytes;
+    unsigned long long off[6];
+    const float* tscale;
+    const uint32_t* need;
+    const uint32_t* ready;
+    float* hbuf;
+    unsigned int* hamax;
+    unsigned int* ctr;
+    int T, k, H, I, E, S, layer, fmt;
+    int RA, RB, stage_bytes, nstage;
+    unsigned long long ready_ns, dep_ns, pipe_ns;
+};
+
+// ------------------------------------------------------------------ helpers
+
+// 16 code bytes = 32 E2M1 elements -> 16 f16x2 words (word i = elements 2i, 2i+1)
+__device__ __forceinline__ void decode_e2m1_16B(const uint4 c, uint32_t (&w)[16]) {
+    const uint32_t v[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int q = 0; q < 4; q++)
+        asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;"
+            " cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;"
+            " cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+            : "=r"(w[4 * q]), "=r"(w[4 * q + 1]), "=r"(w[4 * q + 2]), "=r"(w[4 * q + 3])
+            : "r"(v[q]));
+}
+
+// acc += w.lo * x.lo + w.hi * x.hi, products exact, fp32 accumulation
+__device__ __forceinline__ float fma_f16x2(uint32_t w, uint32_t x, float acc) {
+    asm("{ .reg .f16 wl, wh, xl, xh; mov.b32 {wl, wh}, %1; mov.b32 {xl, xh}, %2;"
+        " fma.rn.f32.f16 %0, wl, xl, %0; fma.rn.f32.f16 %0, wh, xh, %0; }"
+        : "+f"(acc) : "r"(w), "r"(x));
+    return acc;
+}
+
+__device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
+    return e == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23);
+}
+
+// two E4M3 bytes (lo = first block) -> two floats
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two) {
+    uint32_t h2;
+    asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %1; cvt.rn.f16x2.e4m3x2 %0, lo; }"
+        : "=r"(h2) : "r"(two));
+    return make_float2(__half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF))),
+                       __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
+}
+
+// Power-of-two scale putting amax in [2^12, 2^13): bf16 values stay exact in f16
+// and |e2m1 * v| <= 6 * 2^13 stays finite.
+__device__ __forceinline__ float act_scale(float amax) {
+    if (!(amax > 0.0f)) return 1.0f;
+    int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+    int se = 127 + 12 - e;
+    se = se < 1 ? 1 : (se > 254 ? 254 : se);
+    return __uint_as_float((uint32_t)se << 23);
+}
+
+// Dot products of one row chunk (16 code bytes) against MT activation rows.
+// NVFP4: two 16-element blocks per chunk; MXFP4: one 32-element block.
+template <int FMT, int MT>
+__device__ __forceinline__ void chunk_dot(const uint8_t* code, const uint8_t* scl, int c,
+                                          const __half* const* act, int M, float (&acc)[MT]) {
+    uint32_t wv[16];
+    decode_e2m1_16B(*reinterpret_cast<const uint4*>(code + 16 * c), wv);
+    float s0, s1;
+    if (FMT == MOE_NVFP4) {
+        const uint32_t two = (uint32_t)scl[2 * c] | ((uint32_t)scl[2 * c + 1] << 8);
+        const float2 s = e4m3x2_to_f32(two);
+        s0 = s.x;
+        s1 = s.y;
+    } else {
+        s0 = e8m0_to_f32(scl[c]);
+        s1 = s0;
+    }
+#pragma unroll
+    for (int m = 0; m < MT; m++) {
+        if (m >= M) break;
+        const uint4* xp = reinterpret_cast<const uint4*>(act[m] + 32 * c);
+        const uint4 x0 = xp[0], x1 = xp[1], x2 = xp[2], x3 = xp[3];
+        const uint32_t xv[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                 x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+        float p0 = 0.0f, p1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; i++) p0 = fma_f16x2(wv[i], xv[i], p0);
+#pragma unroll
+        for (int i = 8; i < 16; i++) p1 = fma_f16x2(wv[i], xv[i], p1);
+        if (FMT == MOE_NVFP4) {
+            acc[m] = fmaf(p0, s0, acc[m]);
+            acc[m] = fmaf(p1, s1, acc[m]);
+        } else {
+            acc[m] = fmaf(p0 + p1, s0, acc[m]);
+        }
+    }
+}
+
+template <int MT>
+__device__ __forceinline__ void group_reduce(float (&acc)[MT], int G) {
+#pragma unroll
+    for (int m = 0; m < MT; m++)
+        for (int off = G >> 1; off >= 1; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+}
+
+__host__ __device__ __forceinline__ int lanes_per_row(int K) {
+    const int cpr = K / 32;  // 16-byte chunks per row
+    int g = 32;
+    while (g > 1 && cpr % g) g >>= 1;
+    return g;
+}
+
+struct StageMap {  // byte offsets of an item's tensors inside its stage
+    uint32_t codes0, scl0, codes1, scl1;     // A: gate codes/scales, up codes/scales; B: down
+    uint32_t scl0_in, scl1_in;               // start of the rows' scales inside the window
+    uint32_t bytes;
+};
+
+__device__ __forceinline__ void window(unsigned long long start, unsigned long long len,
+                                       unsigned long long& wstart, uint32_t& wlen, uint32_t& in) {
+    wstart = start & ~15ull;
+    in = (uint32_t)(start - wstart);
+    wlen = (uint32_t)(((start + len + 15) & ~15ull) - wstart);
+}
+
+__device__ __forceinline__ bool wait_ready(const FfnArgs& a, int slot, volatile unsigned int* abort_flag) {
+    const uint32_t want = a.need[slot];
+    if (ld_acquire_sys_u32(a.ready + slot) == want) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (ld_acquire_sys_u32(a.ready + slot) == want) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > a.ready_ns) return false;
+        __nanosleep(200);
+    }
+}
+
+template <int FMT, int MT>
+__global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + a.nstage;
+    Group* groups = reinterpret_cast<Group*>(smem + 16 * a.nstage);
+    float* xinv = reinterpret_cast<float*>(groups + kMaxDecodePairs);   // [16]
+    float* hinv = xinv + kMaxDecodeT;                                   // [16]
+    int* s_misc = reinterpret_cast<int*>(hinv + kMaxDecodeT);           // [4]
+    __half* xs = reinterpret_cast<__half*>(
+        (reinterpret_cast<uintptr_t>(s_misc + 4) + 15) & ~uintptr_t(15));  // [T][H]
+    __half* hs = xs + a.T * a.H;                                        // [MT][I]
+    uint8_t* stages = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(hs + MT * a.I) + 127) & ~uintptr_t(127));
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    volatile unsigned int* abort_flag = a.ctr + kAbortIdx;
+    const int bs = FMT == MOE_MXFP4 ? 32 : 16;
+    const unsigned long long codeA = (unsigned long long)a.H / 2, sclA = (unsigned long long)a.H / bs;
+    const unsigned long long codeB = (unsigned long long)a.I / 2, sclB = (unsigned long long)a.I / bs;
+
+    // ---- prologue: barriers, groups, activations
+    if (tid == 0) {
+        for (int i = 0; i < a.nstage; i++) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kNC);
+        }
+        fence_mbar_init();
+        int ng = 0, bad = 0;
+        const int n = a.T * a.k;
+        for (int i = 0; i < n; i++) {
+            const int e = a.idx[i], s = a.slot_of[i];
+            if (e < 0 || e >= a.E) { bad |= MOE_STATUS_BAD_EXPERT; continue; }
+            if (s < 0 || s >= a.S) { bad |= MOE_STATUS_BAD_SLOT; continue; }
+            int g = 0;
+            while (g < ng && groups[g].expert != e) g++;
+            if (g == ng) {
+                groups[g].expert = e;
+                groups[g].slot = s;
+                groups[g].M = 0;
+                const float* ts = a.tscale + ((size_t)a.layer * a.E + e) * 3;
+                groups[g].ts[0] = ts[0];
+                groups[g].ts[1] = ts[1];
+                groups[g].ts[2] = ts[2];
+                ng++;
+            }
+            Group& G = groups[g];
+            G.tok[G.M] = (uint8_t)(i / a.k);
+            G.rank[G.M] = (uint8_t)(i % a.k);
+            G.M++;
+        }
+        // ascending ticket the slot must show: resident experts first, misses in copy order
+        for (int i = 1; i < ng; i++) {
+            Group key = groups[i];
+            const uint32_t kt = a.need[key.slot];
+            int j = i - 1;
+            while (j >= 0 && (a.need[groups[j].slot] > kt ||
+                              (a.need[groups[j].slot] == kt && groups[j].expert > key.expert))) {
+                groups[j + 1] = groups[j];
+                j--;
+            }
+            groups[j + 1] = key;
+        }
+        int pos = 0;
+        for (int g = 0; g < ng; g++) {
+            groups[g].pos = pos;
+            pos += groups[g].M;
+        }
+        s_misc[0] = ng;
+        if (bad && blockIdx.x == 0) atomicOr(a.status, bad);
+    }
+    // activations: per-token power-of-two scale, f16
+    for (int t = warp; t < a.T; t += kNC + 1) {
+        float amax = 0.0f;
+        for (int h = lane; h < a.H; h += 32)
+            amax = fmaxf(amax, fabsf(__uint_as_float((uint32_t)a.x[(size_t)t * a.H + h] << 16)));
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float sc = act_scale(amax);
+        if (lane == 0) xinv[t] = 1.0f / sc;
+        for (int h = lane; h < a.H; h += 32)
+            xs[t * a.H + h] = __float2half_rn(__uint_as_float((uint32_t)a.x[(size_t)t * a.H + h] << 16) * sc);
+    }
+    __syncthreads();
+
+    const int ng = s_misc[0];
+    const int nA_per = a.I / a.RA, nB_per = a.H / a.RB;
+    const int NA = ng * nA_per, N = NA + ng * nB_per;
+
+    auto stage_map = [&](int item, unsigned long long* src, uint32_t* len, int& nsrc) -> StageMap {
+        StageMap m{};
+        const bool isB = item >= NA;
+        const int g = isB ? (item - NA) / nB_per : item / nA_per;
+        const int rb = isB ? (item - NA) % nB_per : item % nA_per;
+        const unsigned long long base = (unsigned long long)groups[g].slot * a.block_bytes;
+        if (!isB) {
+            const unsigned long long r0 = (unsigned long long)rb * a.RA;
+            unsigned long long ws;
+            uint32_t wl, in;
+            m.codes0 = 0;
+            src[0] = base + a.off[0] + r0 * codeA;
+            len[0] = (uint32_t)(a.RA * codeA);
+            window(base + a.off[1] + r0 * sclA, a.RA * sclA, ws, wl, in);
+            m.scl0 = len[0];
+            m.scl0_in = in;
+            src[1] = ws;
+            len[1] = wl;
+            m.codes1 = m.scl0 + wl;
+            src[2] = base + a.off[2] + r0 * codeA;
+            len[2] = len[0];
+            window(base + a.off[3] + r0 * sclA, a.RA * sclA, ws, wl, in);
+            m.scl1 = m.codes1 + len[2];
+            m.scl1_in = in;
+            src[3] = ws;
+            len[3] = wl;
+            m.bytes = m.scl1 + wl;
+            nsrc = 4;
+        } else {
+            const unsigned long long r0 = (unsigned long long)rb * a.RB;
+            unsigned long long ws;
+            uint32_t wl, in;
+            m.codes0 = 0;
+            src[0] = base + a.off[4] + r0 * codeB;
+            len[0] = (uint32_t)(a.RB * codeB);
+            window(base + a.off[5] + r0 * sclB, a.RB * sclB, ws, wl, in);
+            m.scl0 = len[0];
+            m.scl0_in = in;
+            src[1] = ws;
+            len[1] = wl;
+            m.bytes = m.scl0 + wl;
+            nsrc = 2;
+        }
+        return m;
+    };
+
+    if (warp == kNC) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            int it = 0;
+            for (int item = blockIdx.x; item < N; item += gridDim.x, it++) {
+                const int st = it % a.nstage, round = it / a.nstage;
+                if (!mbar_wait(&empty[st], (round & 1) ^ 1, a.pipe_ns)) {
+                    atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                const int g = item >= NA ? (item - NA) / nB_per : item / nA_per;
+                if (!wait_ready(a, groups[g].slot, abort_flag)) {
+                    atomicOr(a.status, MOE_STATUS_READY_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                fence_proxy_async_global();
+                unsigned long long src[4];
+                uint32_t len[4];
+                int nsrc = 0;
+                const StageMap m = stage_map(item, src, len, nsrc);
+                uint8_t* dst = stages + (size_t)st * a.stage_bytes;
+                mbar_arrive_expect_tx(&full[st], m.bytes);
+                uint32_t o = 0;
+                for (int i = 0; i < nsrc; i++) {
+                    bulk_g2s(dst + o, a.slots + src[i], len[i], &full[st]);
+                    o += len[i];
+                }
+            }
+            // no copy may still be in flight when the CTA exits: wait (bounded) for
+            // the last phase of every stage used
+            for (int j = (it > a.nstage ? it - a.nstage : 0); j < it; j++)
+                if (!mbar_wait(&full[j % a.nstage], (j / a.nstage) & 1, a.pipe_ns))
+                    atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
+        }
+    } else {
+        // ---------------------------------------------------------------- consumers
+        const int GA = lanes_per_row(a.H), GB = lanes_per_row(a.I);
+        int it = 0;
+        for (int item = blockIdx.x; item < N; item += gridDim.x, it++) {
+            const int st = it % a.nstage, round = it / a.nstage;
+            const bool ok = mbar_wait(&full[st], round & 1, a.pipe_ns);
+            if (!ok) {
+                if (lane == 0) atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
+                *abort_flag = 1;
+            }
+            unsigned long long src[4];
+            uint32_t len[4];
+            int nsrc;
+            const StageMap m = stage_map(item, src, len, nsrc);
+            const uint8_t* sb = stages + (size_t)st * a.stage_bytes;
+            const bool isB = item >= NA;
+            const int g = isB ? (item - NA) / nB_per : item / nA_per;
+            const Group& G = groups[g];
+            const int M = G.M;
+            if (!isB) {
+                // A: gate row p and up row p of this item per lane group
+                const int rb = item % nA_per;
+                const int RW = 32 / GA, sub = lane / GA, gl = lane % GA;
+                const __half* act[MT];
+#pragma unroll
+                for (int q = 0; q < MT; q++) act[q] = xs + (size_t)G.tok[q < M ? q : 0] * a.H;
+                int rows_done = 0;
+                for (int base = 0; base < a.RA; base += kNC * RW) {
+                    const int p = base + warp * RW + sub;
+                    float ag[MT], au[MT];
+#pragma unroll
+                    for (int q = 0; q < MT; q++) ag[q] = au[q] = 0.0f;
+                    if (p < a.RA && ok) {
+                        const uint8_t* gc = sb + m.codes0 + (size_t)p * codeA;
+                        const uint8_t* gs = sb + m.scl0 + m.scl0_in + (size_t)p * sclA;
+                        const uint8_t* uc = sb + m.codes1 + (size_t)p * codeA;
+                        const uint8_t* us = sb + m.scl1 + m.scl1_in + (size_t)p * sclA;
+                        for (int c = gl; c < (int)(codeA / 16); c += GA) {
+                            chunk_dot<FMT, MT>(gc, gs, c, act, M, ag);
+                            chunk_dot<FMT, MT>(uc, us, c, act, M, au);
+                        }
+                    }
+                    group_reduce<MT>(ag, GA);
+                    group_reduce<MT>(au, GA);
+                    if (p < a.RA && gl == 0) {
+                        const int i = rb * a.RA + p;
+#pragma unroll
+                        for (int q = 0; q < MT; q++) {
+                            if (q >= M) break;
+                            const float xi = xinv[G.tok[q]];
+                            const float gv = ag[q] * xi * G.ts[0];
+                            const float uv = au[q] * xi * G.ts[1];
+                            const float hv = gv / (1.0f + expf(-gv)) * uv;
+                            a.hbuf[(size_t)(G.pos + q) * a.I + i] = hv;
+                            atomicMax(a.hamax + G.pos + q, __float_as_uint(fabsf(hv)));
+                        }
+                        rows_done++;
+                    }
+                }
+                // publish: every writer fences, the warp syncs, lane 0 bumps the counter
+                __threadfence();
+                __syncwarp();
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) rows_done += __shfl_xor_sync(0xffffffffu, rows_done, off);
+                if (lane == 0 && rows_done) {
+                    __threadfence();
+                    atomicAdd(a.ctr + g, (unsigned int)rows_done);
+                }
+            } else {
+                // B: wait for all I rows of h, stage it in f16, then RB rows of down
+                const int rb = (item - NA) % nB_per;
+                if (warp == 0 && lane == 0) {
+                    const unsigned int want = (unsigned int)a.I;
+                    if (ld_acquire_u32(a.ctr + g) < want) {
+                        const unsigned long long t0 = globaltimer();
+                        while (ld_acquire_u32(a.ctr + g) < want) {
+                            if (*abort_flag || globaltimer() - t0 > a.dep_ns) {
+                                atomicOr(a.status, MOE_STATUS_DEP_TIMEOUT);
+                                *abort_flag = 1;
+                                break;
+                            }
+                            __nanosleep(100);
+                        }
+                    }
+                }
+                named_sync(1, kNC * 32);
+                __threadfence();
+                for (int q = warp; q < M; q += kNC) {
+                    const float amax = __uint_as_float(__ldcg(a.hamax + G.pos + q));
+                    const float sc = act_scale(amax);
+                    if (lane == 0) hinv[q] = 1.0f / sc;
+                    const float* hrow = a.hbuf + (size_t)(G.pos + q) * a.I;
+                    for (int i = lane; i < a.I; i += 32) hs[q * a.I + i] = __float2half_rn(__ldcg(hrow + i) * sc);
+                }
+                named_sync(1, kNC * 32);
+                const int RW = 32 / GB, sub = lane / GB, gl = lane % GB;
+                const __half* act[MT];
+#pragma unroll
+                for (int q = 0; q < MT; q++) act[q] = hs + (size_t)(q < M ? q : 0) * a.I;
+                for (int base = 0; base < a.RB; base += kNC * RW) {
+                    const int r = base + warp * RW + sub;
+                    float ay[MT];
+#pragma unroll
+                    for (int q = 0; q < MT; q++) ay[q] = 0.0f;
+                    if (r < a.RB && ok) {
+                        const uint8_t* dc = sb + m.codes0 + (size_t)r * codeB;
+                        const uint8_t* ds = sb + m.scl0 + m.scl0_in + (size_t)r * sclB;
+                        for (int c = gl; c < (int)(codeB / 16); c += GB) chunk_dot<FMT, MT>(dc, ds, c, act, M, ay);
+                    }
+                    group_reduce<MT>(ay, GB);
+                    if (r < a.RB && gl == 0) {
+                        const int row = rb * a.RB + r;
+#pragma unroll
+                        for (int q = 0; q < MT; q++) {
+                            if (q >= M) break;
+                            const int t = G.tok[q], j = G.rank[q];
+                            const float wt = a.w[t * a.k + j];
+                            a.y_part[((size_t)t * a.k + j) * a.H + row] = wt * (ay[q] * hinv[q] * G.ts[2]);
+                        }
+                    }
+                }
+                named_sync(1, kNC * 32);  // hs is rewritten by the next B item
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+    }
+
+    // ---- epilogue: the last CTA clears the per-call counters
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned int prev = atomicAdd(a.ctr + kDoneIdx, 1u);
+        if (prev == gridDim.x - 1) {
+            __threadfence();
+            for (int g = 0; g < ng; g++) a.ctr[g] = 0;
+            for (int i = 0; i < a.T * a.k; i++) a.hamax[i] = 0;
+            a.ctr[kAbortIdx] = 0;
+            a.ctr[kDoneIdx] = 0;
+            __threadfence();
+        }
+    }
+}
+
+// ------------------------------------------------------------------ combine
+
+__global__ void combine_kernel(const float* __restrict__ y_part, int T, int k, int H, uint16_t* __restrict__ y) {
+    const size_t n4 = (size_t)T * H / 4;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t e = i * 4;
+        const size_t t = e / H, h = e % H;
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; j++) {
+            const float4 v = *reinterpret_cast<const float4*>(y_part + (t * k + j) * H + h);
+            s.x += v.x;
+            s.y += v.y;
+            s.z += v.z;
+            s.w += v.w;
+        }
+        const float f[4] = {s.x, s.y, s.z, s.w};
+        uint16_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) o[q] = __bfloat16_as_ushort(__float2bfloat16_rn(f[q]));
+        *reinterpret_cast<uint2*>(y + e) = make_uint2(o[0] | ((uint32_t)o[1] << 16), o[2] | ((uint32_t)o[3] << 16));
+    }
+}
+
+// ------------------------------------------------------------------ dequant
+
+template <int FMT>
+__global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                               float ts, int rows, int K, float* __restrict__ out) {
+    const int bs = FMT == MOE_MXFP4 ? 32 : 16;
+    const size_t nbytes = (size_t)rows * K / 2;
+    for (size_t b = blockIdx.x * (size_t)blockDim.x + threadIdx.x; b < nbytes; b += (size_t)gridDim.x * blockDim.x) {
+        const size_t r = b / (K / 2), c = (b % (K / 2)) * 2;
+        uint32_t h2;
+        asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"((uint32_t)codes[b]));
+        const uint8_t s = scales[r * (K / bs) + c / bs];
+        float sv;
+        if (FMT == MOE_NVFP4) sv = e4m3x2_to_f32((uint32_t)s).x;
+        else sv = e8m0_to_f32(s);
+        float v0 = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF))) * sv;
+        float v1 = __half2float(__ushort_as_half((unsigned short)(h2 >> 16))) * sv;
+        if (FMT == MOE_NVFP4) {
+            v0 *= ts;
+            v1 *= ts;
+        }
+        out[r * K + c] = v0;
+        out[r * K + c + 1] = v1;
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+struct FfnPlan {
+    int RA, RB, stage_bytes, nstage, smem, grid;
+};
+
+static int pick_pow2_rows(int limit_rows, int rows_total, int cap) {
+    int r = 1;
+    while (r * 2 <= cap && r * 2 <= limit_rows && rows_total % (r * 2) == 0) r *= 2;
+    return r;
+}
+
+template <int FMT, int MT>
+static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
+    const moe_config& c = p->cfg;
+    const int bs = p->bs;
+    const size_t rowA = (size_t)c.H / 2 + (size_t)c.H / bs;   // one gate (or up) row
+    const size_t rowB = (size_t)c.I / 2 + (size_t)c.I / bs;
+    // items of about 20 KB, but at least one row (pair) per consumer lane group
+    const size_t target = 20 * 1024;
+    const int minA = kNC * (32 / lanes_per_row(c.H)), minB = kNC * (32 / lanes_per_row(c.I));
+    a.RA = pick_pow2_rows(std::max((int)(target / (2 * rowA)), minA), c.I, 64);
+    a.RB = pick_pow2_rows(std::max((int)(target / rowB), minB), c.H, 256);
+    const size_t bytesA = 2 * ((size_t)a.RA * c.H / 2 + (((size_t)a.RA * c.H / bs + 15) / 16 + 1) * 16);
+    const size_t bytesB = (size_t)a.RB * c.I / 2 + (((size_t)a.RB * c.I / bs + 15) / 16 + 1) * 16;
+    a.stage_bytes = (int)((std::max(bytesA, bytesB) + 127) / 128 * 128);
+    const size_t fixed = 16 * 16 + sizeof(Group) * kMaxDecodePairs + 4 * (2 * kMaxDecodeT + 4) + 16 +
+                        (size_t)a.T * c.H * 2 + (size_t)MT * c.I * 2 + 128;
+    const size_t budget = 227 * 1024;
+    if (fixed + 2 * (size_t)a.stage_bytes > budget) return fail(MOE_EINVAL, "decode FFN: shapes exceed shared memory");
+    a.nstage = (int)std::min<size_t>(12, (budget - fixed) / a.stage_bytes);
+    const size_t smem = 16 * (size_t)a.nstage + sizeof(Group) * kMaxDecodePairs + 4 * (2 * kMaxDecodeT + 4) + 16 +
+                        (size_t)a.T * c.H * 2 + (size_t)MT * c.I * 2 + 128 + (size_t)a.nstage * a.stage_bytes;
+    auto kern = ffn_decode_kernel<FMT, MT>;
+    MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    int per_sm = 0;
+    MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFfnThreads, smem));
+    if (per_sm < 1) return fail(MOE_EINVAL, "decode FFN kernel does not fit on an SM");
+    const int items_max = a.T * a.k * (c.I / a.RA + c.H / a.RB);
+    const int grid = std::max(1, std::min(p->num_sms * per_sm, items_max));
+    void* args[] = {(void*)&a};
+    MOE_CUDA_TRY(cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kFfnThreads), args, smem, s));
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+static unsigned long long g_ready_ns = 5000000000ull, g_dep_ns = 5000000000ull, g_pipe_ns = 10000000000ull;
+
+extern "C" int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms) {
+    if (!(ready_ms > 0) || !(dep_ms > 0) || !(pipe_ms > 0)) return fail(MOE_EINVAL, "wait limits must be positive");
+    g_ready_ns = (unsigned long long)(ready_ms * 1e6);
+    g_dep_ns = (unsigned long long)(dep_ms * 1e6);
+    g_pipe_ns = (unsigned long long)(pipe_ms * 1e6);
+    return MOE_OK;
+}
+
+extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx,
+                              const float* w, const int32_t* slot_of, float* y_part, int* status,
+                              void* stream) {
+    if (!p || !x_bf16 || !idx || !w || !slot_of || !y_part || !status) return fail(MOE_EINVAL, "null argument");
+    const moe_config& c = p->cfg;
+    if (layer < 0 || layer >= c.L) return fail(MOE_EBOUNDS, "layer outside the pool");
+    if (T <= 0 || T > c.max_tokens) return fail(MOE_EINVAL, "decode FFN: T must be in [1, max_tokens]");
+    FfnArgs a{};
+    a.x = (const uint16_t*)x_bf16;
+    a.idx = idx;
+    a.w = w;
+    a.slot_of = slot_of;
+    a.y_part = y_part;
+    a.status = status;
+    a.slots = p->slots;
+    a.block_bytes = p->lay.bytes;
+    for (int i = 0; i < 6; i++) a.off[i] = p->lay.off[i];
+    a.tscale = p->tscale;
+    a.need = p->need;
+    a.ready = p->ready;
+    a.hbuf = p->hbuf;
+    a.hamax = p->hamax;
+    a.ctr = p->ctr;
+    a.T = T;
+    a.k = c.k;
+    a.H = c.H;
+    a.I = c.I;
+    a.E = c.E;
+    a.S = c.n_slots;
+    a.layer = layer;
+    a.fmt = c.fmt;
+    a.ready_ns = g_ready_ns;
+    a.dep_ns = g_dep_ns;
+    a.pipe_ns = g_pipe_ns;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int MT = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16;
+#define DISPATCH(F)                                              \
+    switch (MT) {                                                \
+        case 1: return launch_ffn<F, 1>(p, a, s);                \
+        case 2: return launch_ffn<F, 2>(p, a, s);                \
+        case 4: return launch_ffn<F, 4>(p, a, s);                \
+        case 8: return launch_ffn<F, 8>(p, a, s);                \
+        default: return launch_ffn<F, 16>(p, a, s);              \
+    }
+    if (c.fmt == MOE_NVFP4) { DISPATCH(MOE_NVFP4) } else { DISPATCH(MOE_MXFP4) }
+#undef DISPATCH
+}
+
+extern "C" int moe_combine(const float* y_part, int T, int k, int H, void* y_bf16, void* stream) {
+    if (!y_part || !y_bf16) return fail(MOE_EINVAL, "null argument");
+    if (T <= 0 || k <= 0 || H <= 0 || H % 4) return fail(MOE_EINVAL, "combine: bad shape");
+    const size_t n4 = (size_t)T * H / 4;
+    const int threads = 256;
+    const int blocks = (int)std::min<size_t>((n4 + threads - 1) / threads, 148 * 8);
+    combine_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(y_part, T, k, H, (uint16_t*)y_bf16);
+    MOE_CUDA_TRY(cudaGetLastError());
+    return MOE_OK;
+}
+
+extern "C" int moe_dequant_slot(moe_pool* p, int slot, int key, int which, float* out, void* stream) {
+    if (!p || !out) return fail(MOE_EINVAL, "null argument");
+    const moe_config& c = p->cfg;
+    if (slot < 0 || slot >= c.n_slots || key < 0 || key >= c.L * c.E || which < 0 || which > 2)
+        return fail(MOE_EBOUNDS, "dequant: slot/key/which out of range");
+    const int rows = which == 2 ? c.H : c.I, K = which == 2 ? c.I : c.H;
+    const uint8_t* base = p->slots + (size_t)slot * p->lay.bytes;
+    const uint8_t* codes = base + p->lay.off[2 * which];
+    const uint8_t* scales = base + p->lay.off[2 * which + 1];
+    float ts = 1.0f;
+    if (c.fmt == MOE_NVFP4) MOE_CUDA_TRY(cudaMemcpy(&ts, p->tscale + (size_t)key * 3 + which, 4, cudaMemcpyDeviceToHost));
+    const size_t nbytes = (size_t)rows * K / 2;
+    const int blocks = (int)std::min<size_t>((nbytes + 255) / 256, 148 * 16);
+    if (c.fmt == MOE_NVFP4)
+        dequant_kernel<MOE_NVFP4><<<blocks, 256, 0, (cudaStream_t)stream>>>(codes, scales, ts, rows, K, out);
+    else
+        dequant_kernel<MOE_MXFP4><<<blocks, 256, 0, (cudaStream_t)stream>>>(codes, scales, ts, rows, K, out);
+    MOE_CUDA_TRY(cudaGetLastError());
+    return MOE_OK;
+}

@@ -1,0 +1,206 @@
+// K1 router: logits in a fixed fp32 order, then top-k and routing weights.
+//
+// Each warp owns EPW experts and a tile of TT tokens.  Lane j accumulates, by
+// fmaf in ascending h, the 8-element chunks c with c % 32 == j (16-byte,
+// warp-coalesced loads of W_r; x staged in shared memory as fp32); the 32 lane
+// sums are added by a xor butterfly (16, 8, 4, 2, 1) and the bias is added
+// last.  That order is part of the contract: any implementation following it
+// gets bit-identical logits, hence identical expert indices.
+//
+// The last CTA to finish a token tile (an atomic ticket per tile, reset by that
+// CTA) selects the top-k of each token with one warp (descending logit, ties to
+// the lower index) and writes the softmax weights.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kRouterWarps = 4;
+constexpr int kRouterTileMax = 8;
+
+template <int EPW, int TT>
+__global__ void __launch_bounds__(kRouterWarps * 32)
+router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr,
+              const float* __restrict__ bias, int T, int H, int E, int k, int renorm,
+              int32_t* __restrict__ idx, float* __restrict__ wout, float* __restrict__ logits,
+              unsigned int* __restrict__ tile_cnt) {
+    extern __shared__ float xs[];  // [TT][H] fp32
+    __shared__ int s_last;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t0 = blockIdx.y * TT;
+    const int nt = min(TT, T - t0);
+
+    for (int i = threadIdx.x; i < TT * H; i += blockDim.x) {
+        const int t = i / H;
+        const uint32_t b = t < nt ? x[size_t(t0 + t) * H + (i - t * H)] : 0;
+        xs[i] = __uint_as_float(b << 16);
+    }
+    __syncthreads();
+
+    const int e0 = (blockIdx.x * kRouterWarps + warp) * EPW;
+    float acc[EPW][TT];
+#pragma unroll
+    for (int a = 0; a < EPW; a++)
+#pragma unroll
+        for (int t = 0; t < TT; t++) acc[a][t] = 0.0f;
+
+    const int nchunk = H / 8;
+    for (int c = lane; c < nchunk; c += 32) {
+        float wf[EPW][8];
+#pragma unroll
+        for (int a = 0; a < EPW; a++) {
+            const int e = e0 + a;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (e < E) v = __ldg(reinterpret_cast<const uint4*>(wr + size_t(e) * H) + c);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                wf[a][2 * q] = __uint_as_float(u[q] << 16);
+                wf[a][2 * q + 1] = __uint_as_float(u[q] & 0xFFFF0000u);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < TT; t++) {
+            const float4 xa = *reinterpret_cast<const float4*>(xs + t * H + c * 8);
+            const float4 xb = *reinterpret_cast<const float4*>(xs + t * H + c * 8 + 4);
+            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int a = 0; a < EPW; a++)
+#pragma unroll
+                for (int q = 0; q < 8; q++) acc[a][t] = fmaf(xv[q], wf[a][q], acc[a][t]);
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < EPW; a++)
+#pragma unroll
+        for (int t = 0; t < TT; t++) {
+            float v = acc[a][t];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, off);
+            const int e = e0 + a;
+            if (lane == 0 && e < E && t < nt)
+                logits[size_t(t0 + t) * E + e] = v + (bias ? bias[e] : 0.0f);
+        }
+
+    // last CTA of this token tile does the selection
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned int prev = atomicAdd(tile_cnt + blockIdx.y, 1u);
+        s_last = (prev == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    __shared__ float s_l[kRouterWarps][kMaxE];
+    __shared__ unsigned char s_taken[kRouterWarps][kMaxE];
+    for (int t = warp; t < nt; t += kRouterWarps) {
+        const float* row = logits + size_t(t0 + t) * E;
+        for (int e = lane; e < E; e += 32) {
+            s_l[warp][e] = __ldcg(row + e);
+            s_taken[warp][e] = 0;
+        }
+        __syncwarp();
+        float my_l = 0.0f;
+        int my_e = -1;
+        for (int j = 0; j < k; j++) {
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+            for (int e = lane; e < E; e += 32) {
+                const float v = s_l[warp][e];
+                if (!s_taken[warp][e] && (v > bv || (v == bv && e < be) || be == 0x7fffffff)) {
+                    bv = v;
+                    be = e;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            if (lane == 0) s_taken[warp][be] = 1;
+            if (lane == j) {
+                my_l = bv;
+                my_e = be;
+            }
+            __syncwarp();
+        }
+        const float lmax = __shfl_sync(0xffffffffu, my_l, 0);
+        float den = 0.0f;
+        if (renorm) {
+            den = lane < k ? expf(my_l - lmax) : 0.0f;
+        } else {
+            for (int e = lane; e < E; e += 32) den += expf(s_l[warp][e] - lmax);
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+        if (lane < k) {
+            idx[size_t(t0 + t) * k + lane] = my_e;
+            wout[size_t(t0 + t) * k + lane] = expf(my_l - lmax) / den;
+        }
+        __syncwarp();
+    }
+    if (threadIdx.x == 0) tile_cnt[blockIdx.y] = 0;
+}
+
+static size_t round_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
+
+template <int EPW, int TT>
+static cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const float* bias, int T,
+                                 int H, int E, int k, int renorm, int32_t* idx, float* w,
+                                 float* logits, unsigned int* cnt, cudaStream_t s) {
+    const size_t smem = size_t(TT) * H * sizeof(float);
+    auto kern = router_kernel<EPW, TT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((E + kRouterWarps * EPW - 1) / (kRouterWarps * EPW), (T + TT - 1) / TT);
+    kern<<<grid, kRouterWarps * 32, smem, s>>>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt);
+    return cudaGetLastError();
+}
+
+// Shared by the entry points that own their scratch differently.
+int route_impl(const void* x_bf16, const void* wr_bf16, const float* bias, int T, int H, int E,
+               int k, int renorm, int32_t* idx, float* w, float* logits, unsigned int* cnt,
+               cudaStream_t s) {
+    if (!x_bf16 || !wr_bf16 || !idx || !w || !logits || !cnt) return fail(MOE_EINVAL, "null pointer");
+    if (T <= 0 || H <= 0 || H % 256 || E <= 0 || E > kMaxE || k <= 0 || k > kMaxK || k > E)
+        return fail(MOE_EINVAL, "route: need T > 0, H % 256 == 0, 0 < k <= min(E, 32), E <= 1024");
+    if (size_t(kRouterTileMax) * H * sizeof(float) > 200 * 1024)
+        return fail(MOE_EINVAL, "route: H too large for the shared-memory x tile");
+    const uint16_t* x = (const uint16_t*)x_bf16;
+    const uint16_t* wr = (const uint16_t*)wr_bf16;
+    cudaError_t e;
+    if (T == 1) e = launch_router<1, 1>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt, s);
+    else if (T == 2) e = launch_router<1, 2>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt, s);
+    else if (T <= 4) e = launch_router<1, 4>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt, s);
+    else if (T <= 8) e = launch_router<2, 8>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt, s);
+    else e = launch_router<4, 8>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt, s);
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    return MOE_OK;
+}
+
+size_t route_logits_bytes(int T, int E) { return round_up(size_t(T) * E * sizeof(float), 256); }
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t moe_route_workspace_bytes(int T, int E) {
+    if (T <= 0 || E <= 0) return 0;
+    return route_logits_bytes(T, E) + round_up(size_t((T + kRouterTileMax - 1) / kRouterTileMax) * 4, 256);
+}
+
+extern "C" int moe_route(const void* x_bf16, const void* wr_bf16, const float* bias, int T, int H,
+                         int E, int k, int renormalize, int32_t* idx, float* w, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < moe_route_workspace_bytes(T, E))
+        return fail(MOE_EINVAL, "route: workspace missing or smaller than moe_route_workspace_bytes");
+    float* logits = (float*)workspace;
+    unsigned int* cnt = (unsigned int*)((char*)workspace + route_logits_bytes(T, E));
+    return route_impl(x_bf16, wr_bf16, bias, T, H, E, k, renormalize, idx, w, logits, cnt,
+                      (cudaStream_t)stream);
+}

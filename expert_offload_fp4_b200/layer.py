@@ -1,0 +1,42 @@
+"""One decode MoE layer through the C ABI: route -> slot lookup -> miss
+streaming (copy stream) -> expert FFN (compute stream) -> combine.
+
+This is the public call a user makes per (token batch, layer); it owns only the
+per-call device buffers.  The copy of missed experts runs on its own stream and
+the FFN kernel starts at once: CTAs on resident experts compute while the copy
+engine streams the misses, whose CTAs wait for the slot's ready ticket.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import api
+
+
+class DecodeLayer:
+    def __init__(self, pool: api.Pool, T: int, device="cuda", renormalize=1):
+        if T > pool.max_tokens:
+            raise ValueError("T exceeds the pool's max_tokens")
+        self.pool, self.T, self.renormalize = pool, T, renormalize
+        k, H, E = pool.k, pool.H, pool.E
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.slot_of = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.y_part = torch.empty((T, k, H), dtype=torch.float32, device=device)
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ws = torch.zeros(api.route_workspace_bytes(T, E), dtype=torch.uint8, device=device)
+        self.lookup = api.Lookup(min(T * k, E))
+        self.copy_stream = torch.cuda.Stream(device=device)
+
+    def __call__(self, layer, x, wr, bias, stream=None):
+        """x [T, H] bf16, wr [E, H] bf16, bias [E] fp32 (or None), all on the device.
+        Returns y [T, H] bf16 (a buffer reused by the next call)."""
+        p = self.pool
+        api.route(x, wr, bias, p.k, self.renormalize, self.idx, self.w, self.ws, stream)
+        api.slot_lookup(p, layer, self.idx, self.slot_of, self.lookup, stream)
+        if self.lookup.n_miss:
+            api.stream_misses(p, layer, self.lookup, self.copy_stream)
+        api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, stream)
+        api.combine(self.y_part, self.y, stream)
+        return self.y

@@ -1,0 +1,217 @@
+/*
+ * moe_fp4.h -- C ABI of the B200 (sm_100a) hot path of one FreeToken-style MoE
+ * layer with FP4 experts offloaded to pinned host memory.
+ *
+ * The layer, per decode step: route each token to k of E experts; look the
+ * chosen experts up in an LRU pool of expert slots held in HBM; stream the
+ * missed experts from pinned host memory into their slots on the copy engine
+ * while the hits are already being computed; run the SwiGLU expert FFN on the
+ * FP4 weights; merge the expert outputs by routing weight.  The q* bandwidth
+ * split is a host function whose result is reported (every expert runs on the
+ * GPU here).
+ *
+ * Conventions
+ *  - Every call returns an int status (MOE_OK = 0 or an MOE_E* code); on error
+ *    moe_last_error() returns a message for the calling thread.
+ *  - Pointers are device pointers unless their name ends in _h (host memory).
+ *    Device buffers and streams are owned by the caller; the pool (slot storage
+ *    in HBM, pinned host expert store, slot metadata, scratch) is owned by the
+ *    library and only created / destroyed through moe_pool_create/destroy.
+ *  - A stream is a cudaStream_t passed as void* (NULL = the legacy stream).
+ *  - Calls are asynchronous on their stream, except moe_slot_lookup, which
+ *    waits (bounded) for the lookup kernel because the host must drive the copy
+ *    engine with the miss list, and the pool create/load/state/stats calls.
+ *  - Tensor layouts (row-major, "canonical"): bf16 activations x [T, H];
+ *    router weight W_r [E, H] bf16; FP4 codes [rows, K/2] bytes with element c
+ *    of a row in byte c/2, the lower element index in the low nibble; block
+ *    scales [rows, K/bs] bytes, bs = 32 (MXFP4, E8M0) or 16 (NVFP4, E4M3).
+ *    gate and up are [I, H] (K = H), down is [H, I] (K = I).
+ */
+#ifndef MOE_FP4_H
+#define MOE_FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    MOE_OK = 0,
+    MOE_EINVAL = 1,   /* bad argument or shape outside the supported range */
+    MOE_ENOMEM = 2,   /* device or pinned host allocation failed */
+    MOE_ECUDA = 3,    /* a CUDA runtime call failed */
+    MOE_ETIMEOUT = 4, /* a bounded wait (host or device) gave up */
+    MOE_EBOUNDS = 5,  /* an index (layer, expert, slot) outside the pool */
+    MOE_ESTATE = 6    /* call out of order (e.g. expert not loaded) */
+};
+
+/* FP4 expert formats named by the pages (post.smzdm.com/p/a825qpgl, section 一:
+ * MXFP4 expert weights; an NVFP4 build of the 35B-A3B model).  Bit layouts from
+ * the OCP MX v1.0 spec (E2M1 codes, E8M0 scale per 32) and NVIDIA's NVFP4
+ * description (E2M1 codes, E4M3 scale per 16, FP32 tensor scale). */
+enum { MOE_MXFP4 = 0, MOE_NVFP4 = 1 };
+
+/* Bits of the device status word written by moe_expert_ffn. */
+enum {
+    MOE_STATUS_READY_TIMEOUT = 1,  /* a missed expert's ready flag never arrived */
+    MOE_STATUS_DEP_TIMEOUT = 2,    /* down projection waited too long for h */
+    MOE_STATUS_BAD_SLOT = 4,       /* slot index outside the pool */
+    MOE_STATUS_BAD_EXPERT = 8,     /* expert index outside [0, E) */
+    MOE_STATUS_PIPE_TIMEOUT = 16   /* a shared-memory pipeline wait gave up */
+};
+
+typedef struct {
+    int H;            /* hidden size, multiple of 256 */
+    int I;            /* expert intermediate size, multiple of 256 */
+    int E;            /* experts per layer, <= 1024 */
+    int k;            /* experts chosen per token, <= 32 */
+    int L;            /* MoE layers sharing the slot pool */
+    int fmt;          /* MOE_MXFP4 or MOE_NVFP4 */
+    int n_slots;      /* expert slots in HBM, >= the unique experts of one call */
+    int max_tokens;   /* largest T of a decode call (moe_expert_ffn), <= 16 */
+    int host_layers;  /* distinct host copies of the layers: layer l is stored at
+                         l % host_layers (0 means L); lets a large model's host
+                         store be folded when pinned RAM is short */
+    int reserved[3];
+} moe_config;
+
+typedef struct moe_pool moe_pool;
+
+/* One expert in the canonical layout (host memory).  tensor_scale[i] is the
+ * NVFP4 FP32 tensor scale of gate/up/down (ignored for MXFP4). */
+typedef struct {
+    const uint8_t* codes_h[3];   /* gate [I, H/2], up [I, H/2], down [H, I/2] */
+    const uint8_t* scales_h[3];  /* gate [I, H/bs], up [I, H/bs], down [H, I/bs] */
+    float tensor_scale[3];
+} moe_expert_src;
+
+/* One missed expert of a lookup: copy the host block of (layer, expert) into
+ * `slot`, then publish `ticket` in the slot's ready flag. */
+typedef struct {
+    int32_t expert;
+    int32_t slot;
+    uint32_t ticket;
+    int32_t evicted_key;         /* layer*E + expert evicted from the slot, -1 if free */
+} moe_miss;
+
+typedef struct {
+    int n_uniq;                  /* unique experts of the call, ascending id */
+    int n_miss;
+    int32_t* uniq_h;             /* caller array, capacity >= min(T*k, E) */
+    int32_t* is_hit_h;           /* caller array, same capacity */
+    moe_miss* miss_h;            /* caller array, same capacity */
+} moe_lookup_result;
+
+typedef struct {
+    long long lookups, unique, hits, misses, evictions;
+    long long h2d_bytes, h2d_copies;
+} moe_stats;
+
+const char* moe_last_error(void);
+
+/* ---------------------------------------------------------------- the pool */
+
+/* The expert store in the 4096-byte aligned per-expert layout ("FTW": every
+ * tensor 4096-aligned so that a miss is one large DMA; "跑不快大模型，先别急着怪
+ * 显卡", section 三) and the HBM slot pool.  Block = [gate codes][gate scales]
+ * [up codes][up scales][down codes][down scales], each padded to 4096 bytes;
+ * the FP32 tensor scales stay resident in a small HBM table.  Allocates
+ * n_slots blocks of HBM (cudaMalloc) and host_layers*E blocks of pinned host
+ * memory (cudaHostAlloc).  Errors: MOE_EINVAL (shape), MOE_ENOMEM. */
+int moe_pool_create(const moe_config* cfg, moe_pool** out);
+int moe_pool_destroy(moe_pool* pool);
+size_t moe_expert_block_bytes(const moe_config* cfg);
+
+/* Pack one expert from the canonical layout into its pinned host block.  The
+ * expert is not resident until a lookup misses it.  Errors: MOE_EBOUNDS. */
+int moe_pool_load_expert(moe_pool* pool, int layer, int expert, const moe_expert_src* src);
+
+/* Copy the LRU state to host arrays (synchronous; for checks and checkpoints):
+ * slot_key_h[n_slots] (layer*E+expert or -1), slot_clock_h[n_slots],
+ * key_slot_h[L*E] (slot or -1), *clock_h = global clock. */
+int moe_pool_read_state(moe_pool* pool, int32_t* slot_key_h, uint64_t* slot_clock_h,
+                        int32_t* key_slot_h, uint64_t* clock_h);
+int moe_pool_stats(const moe_pool* pool, moe_stats* out);
+/* Device pointer and byte size of one slot (for checks). */
+int moe_pool_slot_ptr(moe_pool* pool, int slot, void** ptr, size_t* bytes);
+
+/* ---------------------------------------------------------------- the path */
+
+/* Router (mubeitech "游戏电脑如何跑动2840亿参数大模型": the gate picks a few
+ * experts per token; post.smzdm.com/p/a825qpgl section 二: 256 experts, 6
+ * active).  logits[t,e] = sum_h x[t,h]*W_r[e,h] + bias[e] in fp32 with a fixed
+ * order (lane j of 32 accumulates, by fmaf in ascending h, the 8-element chunks
+ * c with c%32 == j; lanes are added by a xor-butterfly 16,8,4,2,1; then +bias),
+ * top-k by descending logit with ties to the lower index, and
+ * w = softmax over the k chosen (renormalize=1) or the full softmax read at the
+ * chosen experts (renormalize=0).  bias may be NULL.  Outputs idx [T,k] int32
+ * and w [T,k] fp32 in rank order.  workspace: device scratch of
+ * moe_route_workspace_bytes(T, E) bytes, its counters zero before the first
+ * use (the call leaves them zero).  Limits: H % 256 == 0, E <= 1024,
+ * k <= min(E, 32).  Errors: MOE_EINVAL. */
+size_t moe_route_workspace_bytes(int T, int E);
+int moe_route(const void* x_bf16, const void* wr_bf16, const float* bias, int T, int H, int E,
+              int k, int renormalize, int32_t* idx, float* w, void* workspace,
+              size_t workspace_bytes, void* stream);
+
+/* LRU slot lookup (post.smzdm.com/p/aomxznrn, "FreeToken干的事": a global LRU
+ * expert-slot pool).  One kernel, one CTA: the unique experts of idx in
+ * ascending id; hits are touched first (clock = ++G), then each miss takes the
+ * lowest free slot, else the occupied slot not used by this call with the
+ * oldest clock; a miss gets clock = ++G and a ticket.  Writes slot_of [T,k]
+ * (device) and, after a bounded wait for the kernel (MOE_ETIMEOUT), fills
+ * *res (host).  The pool must hold at least the call's unique experts. */
+int moe_slot_lookup(moe_pool* pool, int layer, const int32_t* idx, int T, int k, int32_t* slot_of,
+                    moe_lookup_result* res, void* stream);
+
+/* Miss streaming ("游戏电脑如何跑动2840亿参数大模型": prefetch with a double
+ * buffer, copies in the background while computing).  For each miss, in order,
+ * one cudaMemcpyAsync of the expert's pinned host block into its slot on
+ * copy_stream, then a stream write of the ticket into the slot's ready flag.
+ * moe_expert_ffn starts at once on another stream; its CTAs on missed experts
+ * wait (bounded) for the flag, so the copy of miss j+1 overlaps compute on the
+ * hits and on miss j.  Errors: MOE_EBOUNDS, MOE_ESTATE (expert never loaded). */
+int moe_stream_misses(moe_pool* pool, int layer, const moe_miss* miss_h, int n_miss,
+                      void* copy_stream);
+
+/* Decode expert FFN (post.smzdm.com/p/aomxznrn: decode is bandwidth-bound and
+ * scheduled apart from prefill).  For every (t, j): y_part[t, j, :] =
+ * w[t,j] * Wd (silu(Wg x_t) * (Wu x_t)) of expert idx[t,j] read from slot
+ * slot_of[t,j]; FP4 weights dequantised on the fly (MXFP4: e2m1 * 2^(s-127);
+ * NVFP4: e2m1 * e4m3(s) * S_tensor), fp32 accumulation.  One persistent kernel
+ * with a TMA-bulk / shared-memory pipeline; waits are bounded and failures set
+ * bits of *status (device int, caller-zeroed; MOE_STATUS_*).  y_part is
+ * [T, k, H] fp32.  Limits: T <= max_tokens of the pool.  Errors: MOE_EINVAL. */
+int moe_expert_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const int32_t* idx,
+                   const float* w, const int32_t* slot_of, float* y_part, int* status,
+                   void* stream);
+
+/* Limits of the device-side bounded waits of moe_expert_ffn, in milliseconds:
+ * a missed expert's ready flag (default 5000), the down projection's wait for
+ * all rows of h (default 5000), a shared-memory pipeline stage (default 10000).
+ * Process-wide; affects later launches.  Errors: MOE_EINVAL (non-positive). */
+int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
+
+/* Router-weighted combine (post.smzdm.com/p/a825qpgl section 二: results merged
+ * by routing weight): y[t, :] = bf16(sum over j = 0..k-1 of y_part[t, j, :]),
+ * summed in fp32 in rank order, rounded to nearest even. */
+int moe_combine(const float* y_part, int T, int k, int H, void* y_bf16, void* stream);
+
+/* q* split (post.smzdm.com/p/a825qpgl section 二: q* = m*B_p/B_h; "跑不快大模型，
+ * 先别急着怪显卡" section 二: pull : compute = pcie_bw : (cpu_bw - pcie_bw)).
+ * ratio = B_p/B_h; q_gpu = min(m, floor(m*ratio + 0.5)); q_cpu = m - q_gpu.
+ * Host only.  Errors: MOE_EINVAL (m < 0 or a bandwidth <= 0). */
+int qstar_split(int m, double b_pcie, double b_host, int* q_gpu, int* q_cpu, double* ratio);
+
+/* Dequantise tensor `which` (0 gate, 1 up, 2 down) of the expert in `slot`
+ * to fp32 [rows, K] in canonical order: (e2m1(c) * scale) * S_tensor, two fp32
+ * multiplies (the second only for NVFP4).  key = layer*E + expert selects the
+ * tensor scale.  For checks of the slot contents. */
+int moe_dequant_slot(moe_pool* pool, int slot, int key, int which, float* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_FP4_H */

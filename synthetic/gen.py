@@ -189,3 +189,23 @@ def expert_weights(w: Workload, layer: int, expert: int) -> dict:
     assert all(s.shape[1] == (K // block_elems(w.fmt)) for (_, s, _), K in
                zip(out.values(), (w.H, w.H, w.I)))
     return out
+
+
+def _expert_job(args):
+    w, layer, expert = args
+    return expert, expert_weights(w, layer, expert)
+
+
+def expert_weights_many(w: Workload, layer: int, experts, workers: int | None = None) -> dict:
+    """expert_weights for many experts, fanned out over a spawn-started process pool
+    (safe to call after CUDA is initialised in the parent)."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    import os
+    experts = list(experts)
+    if workers is None:
+        workers = min(len(experts), os.cpu_count() or 1, 32)
+    if workers <= 1 or len(experts) <= 2:
+        return {e: expert_weights(w, layer, e) for e in experts}
+    with cf.ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn")) as ex:
+        return dict(ex.map(_expert_job, [(w, layer, e) for e in experts], chunksize=1))
