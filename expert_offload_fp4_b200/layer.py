@@ -28,6 +28,10 @@ class DecodeLayer:
         self.ws = torch.zeros(api.route_workspace_bytes(T, E), dtype=torch.uint8, device=device)
         self.lookup = api.Lookup(min(T * k, E))
         self.copy_stream = torch.cuda.Stream(device=device)
+        # optional timing hooks: lists that receive (start, end) CUDA events recorded
+        # around the FFN launch (compute stream) and around the miss copies (copy stream)
+        self.ffn_events = None
+        self.copy_events = None
 
     def __call__(self, layer, x, wr, bias, stream=None):
         """x [T, H] bf16, wr [E, H] bf16, bias [E] fp32 (or None), all on the device.
@@ -36,7 +40,20 @@ class DecodeLayer:
         api.route(x, wr, bias, p.k, self.renormalize, self.idx, self.w, self.ws, stream)
         api.slot_lookup(p, layer, self.idx, self.slot_of, self.lookup, stream)
         if self.lookup.n_miss:
+            if self.copy_events is not None:
+                ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                ev[0].record(self.copy_stream)
             api.stream_misses(p, layer, self.lookup, self.copy_stream)
+            if self.copy_events is not None:
+                ev[1].record(self.copy_stream)
+                self.copy_events.append((ev, self.lookup.n_miss))
+        if self.ffn_events is not None:
+            cur = stream if stream is not None else torch.cuda.current_stream()
+            fe = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            fe[0].record(cur)
         api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, stream)
+        if self.ffn_events is not None:
+            fe[1].record(cur)
+            self.ffn_events.append((fe, self.lookup.n_uniq, self.lookup.n_miss))
         api.combine(self.y_part, self.y, stream)
         return self.y
