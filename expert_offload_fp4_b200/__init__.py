@@ -5,5 +5,6 @@ bandwidth split.  The work is in libmoe_fp4.so (include/moe_fp4.h); this package
 is its Python binding."""
 from . import _lib  # noqa: F401
 from .api import (Lookup, Pool, combine, dequant_slot, expert_ffn, qstar_split,  # noqa: F401
-                  route, route_workspace_bytes, set_wait_limits, slot_lookup, stream_misses)
+                  route, route_noalloc, route_workspace_bytes, set_wait_limits, slot_lookup,
+                  stream_misses)
 from .layer import DecodeLayer  # noqa: F401

@@ -104,6 +104,15 @@ def route(x, wr, bias, k, renormalize, idx, w, workspace, stream=None):
         _p(workspace), workspace.numel() * workspace.element_size(), _s(stream)))
 
 
+def route_noalloc(x, wr, bias, k, renormalize, idx, w, stream=None):
+    """moe_route_noalloc: the router with its scratch in a static device array of
+    the library (for callers that cannot allocate device memory)."""
+    T, H = x.shape
+    E = wr.shape[0]
+    L.check("moe_route_noalloc", L.load().moe_route_noalloc(
+        _p(x), _p(wr), _p(bias), T, H, E, int(k), int(renormalize), _p(idx), _p(w), _s(stream)))
+
+
 class Lookup:
     """Host-side result of one slot lookup (arrays sized for the call)."""
 

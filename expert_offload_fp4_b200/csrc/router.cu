@@ -204,3 +204,65 @@ extern "C" int moe_route(const void* x_bf16, const void* wr_bf16, const float* b
     return route_impl(x_bf16, wr_bf16, bias, T, H, E, k, renormalize, idx, w, logits, cnt,
                       (cudaStream_t)stream);
 }
+
+// ---------------------------------------------------------------------------
+// Router without allocation.  Some callers cannot allocate device memory where
+// they route: a serving loop that handed every byte of HBM to its KV cache and
+// expert slots at start-up, or code that must not pay cudaMalloc's latency and
+// implicit device-wide synchronisation in the middle of a decode step.  For
+// them the scratch lives in this file-scope array instead of a caller
+// workspace: logits of at most kNoAllocMaxLogits = T*E floats, then one counter
+// per 8-token tile.  Every GPU that loads the library holds the array until the
+// process exits.  All calls share it, and it keeps the last call's contents, so
+// calls that overlap on the GPU race: issue them on one stream, one at a time.
+#include <mutex>
+
+namespace moe {
+
+constexpr int kNoAllocMaxLogits = 1 << 16;   // T*E <= 65536 floats (256 KiB)
+constexpr int kNoAllocMaxT = 4096;           // so at most 512 tile counters
+constexpr size_t kNoAllocLogitBytes = size_t(kNoAllocMaxLogits) * sizeof(float);
+constexpr size_t kNoAllocCounterBytes = size_t(kNoAllocMaxT / kRouterTileMax) * sizeof(unsigned int);
+
+static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocLogitBytes + kNoAllocCounterBytes];
+
+// In host code g_route_scratch names a host-side stand-in, not device memory;
+// the device address is fetched once per device (with that device current).
+constexpr int kMaxDevices = 64;
+static std::mutex g_scratch_mu;
+static void* g_scratch_ptr[kMaxDevices] = {};
+
+static int route_scratch(void** out) {
+    int dev = -1;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_EINVAL, "route_noalloc: device ordinal out of range");
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(route scratch)");
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" int moe_route_noalloc(const void* x_bf16, const void* wr_bf16, const float* bias, int T,
+                                 int H, int E, int k, int renormalize, int32_t* idx, float* w,
+                                 void* stream) {
+    if (T <= 0 || E <= 0 || T > kNoAllocMaxT || (long long)T * E > kNoAllocMaxLogits)
+        return fail(MOE_EINVAL, "route_noalloc: needs 0 < T <= 4096 and T*E <= 65536 "
+                                "(the static scratch holds 65536 logits)");
+    void* base = nullptr;
+    int rc = route_scratch(&base);
+    if (rc) return rc;
+    float* logits = (float*)base;
+    unsigned int* cnt = (unsigned int*)((char*)base + kNoAllocLogitBytes);
+    const int tiles = (T + kRouterTileMax - 1) / kRouterTileMax;
+    // the tile counters must start at zero whatever the previous call left
+    MOE_CUDA_TRY(cudaMemsetAsync(cnt, 0, size_t(tiles) * sizeof(unsigned int), (cudaStream_t)stream));
+    return route_impl(x_bf16, wr_bf16, bias, T, H, E, k, renormalize, idx, w, logits, cnt,
+                      (cudaStream_t)stream);
+}

@@ -156,6 +156,19 @@ int moe_route(const void* x_bf16, const void* wr_bf16, const float* bias, int T,
               int k, int renormalize, int32_t* idx, float* w, void* workspace,
               size_t workspace_bytes, void* stream);
 
+/* Router without allocation (no counterpart in the paper).  The same router as
+ * moe_route, for callers that cannot allocate device memory where they route
+ * (HBM fully handed out at start-up, or no cudaMalloc allowed inside a decode
+ * step): its scratch is a static device array inside the library, so the caller
+ * passes only inputs and outputs.  Limits: T <= 4096 and T*E <= 65536 (256 KiB
+ * of logits), else MOE_EINVAL.  The first call on a device looks the array's
+ * address up; make that first call before any stream capture.  Every call
+ * shares the array: calls that overlap on the GPU race, so serialise them on
+ * one stream.  The array's memory is held on every GPU that loads the library
+ * until the process exits.  Allocates nothing (no cudaMalloc / cudaFree). */
+int moe_route_noalloc(const void* x_bf16, const void* wr_bf16, const float* bias, int T, int H,
+                      int E, int k, int renormalize, int32_t* idx, float* w, void* stream);
+
 /* LRU slot lookup (post.smzdm.com/p/aomxznrn, "FreeToken干的事": a global LRU
  * expert-slot pool).  One kernel, one CTA: the unique experts of idx in
  * ascending id; hits are touched first (clock = ++G), then each miss takes the
