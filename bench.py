@@ -122,6 +122,41 @@ def preload(torch, m, pool, w):
     cs.synchronize()
 
 
+def ffn_roofline(torch, m, w, pool, T, x_dev, wr, bias, reps=4):
+    """Time the decode FFN kernel alone: route and look up all L layers first (all
+    resident, so every expert is a hit), then enqueue reps*L FFN launches back to
+    back behind a device-side sleep (so the host's launch latency stays outside the
+    window) between two CUDA events on the launching stream."""
+    L_ = w.L
+    idx = torch.empty((L_, T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((L_, T, w.k), dtype=torch.float32, device="cuda")
+    slot_of = torch.empty((L_, T, w.k), dtype=torch.int32, device="cuda")
+    y_part = torch.empty((T, w.k, w.H), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(m.route_workspace_bytes(T, w.E), dtype=torch.uint8, device="cuda")
+    uniq = []
+    for l in range(L_):
+        m.route(x_dev[l], wr, bias, w.k, 1, idx[l], wt[l], ws)
+        res = m.slot_lookup(pool, l, idx[l], slot_of[l])
+        assert res.n_miss == 0, "roofline pass expects an all-resident pool"
+        uniq.append(res.n_uniq)
+    for l in range(L_):     # warm-up
+        m.expert_ffn(pool, l, x_dev[l], idx[l], wt[l], slot_of[l], y_part, status)
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(20_000_000)
+    e0.record(cur)
+    for r in range(reps):
+        for l in range(L_):
+            m.expert_ffn(pool, l, x_dev[l], idx[l], wt[l], slot_of[l], y_part, status)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ms = e0.elapsed_time(e1) / (reps * L_)
+    return ms, uniq
+
+
 def expert_bytes_alg(w):
     """Algorithmic HBM bytes of one expert: FP4 codes + block scales of gate, up, down."""
     bs = W.block_elems(w.fmt)
@@ -130,9 +165,9 @@ def expert_bytes_alg(w):
 
 # ---------------------------------------------------------------- decode runs
 
-def decode_run(torch, m, w, pool, T, xs_dev, wr, bias, steps, warmup, events=False):
+def decode_run(torch, m, w, pool, T, xs_dev, wr, bias, steps, warmup, events=False, overlap=True):
     """Times `steps` decode steps (all L layers each) on the current stream."""
-    lo = m.DecodeLayer(pool, T)
+    lo = m.DecodeLayer(pool, T, overlap=overlap)
     cur = torch.cuda.current_stream()
     for s in range(warmup):
         for l in range(w.L):
@@ -158,10 +193,10 @@ def decode_run(torch, m, w, pool, T, xs_dev, wr, bias, steps, warmup, events=Fal
     return out
 
 
-def e2e_run(torch, m, w, pool, T, xs_host, wr, bias, steps, warmup):
+def e2e_run(torch, m, w, pool, T, xs_host, wr, bias, steps, warmup, overlap=True):
     """Through DecodeLayer with x copied in from pinned host memory and every
     layer's y read back to pinned host memory, each step."""
-    lo = m.DecodeLayer(pool, T)
+    lo = m.DecodeLayer(pool, T, overlap=overlap)
     cur = torch.cuda.current_stream()
     nbuf = xs_host.shape[0]
     x_dev = torch.empty(xs_host.shape[1:], dtype=torch.bfloat16, device="cuda")
@@ -214,6 +249,41 @@ def oracle_sample(w, T, experts, budget_s=10.0, min_layers=2):
                        f"{busy:.1f} s on one host core, extrapolated to {w.L} layers")
 
 
+def ffn_only(args, w, T):
+    """The decode FFN kernel alone on `args.layers` all-resident layer positions."""
+    from dataclasses import replace
+    wl = replace(w, L=args.layers)
+    experts = gen.expert_weights_many(wl, 0, range(wl.E))
+    import torch
+    import expert_offload_fp4_b200 as m
+    pool = make_pool(m, wl, wl.L * wl.E, 8, 1, experts)
+    preload(torch, m, pool, wl)
+    xs = np.stack([gen.activations(wl, l, 0, T) for l in range(wl.L)])
+    x_dev = torch.from_numpy(xs.view(np.int16)).cuda().view(torch.bfloat16)
+    wr = torch.from_numpy(gen.router_weight(wl, 0).view(np.int16)).cuda().view(torch.bfloat16)
+    bias = torch.from_numpy(gen.router_bias(wl, 0)).cuda()
+    ms, uniq = ffn_roofline(torch, m, wl, pool, T, x_dev, wr, bias, reps=2)
+    phases = None
+    if args.trace:
+        buf = torch.zeros((148, 8), dtype=torch.int64, device="cuda")
+        m._lib.load().moe_set_ffn_trace(buf.data_ptr())
+        ffn_roofline(torch, m, wl, pool, T, x_dev, wr, bias, reps=1)
+        m._lib.load().moe_set_ffn_trace(None)
+        tr = buf.cpu().numpy().astype(np.float64)
+        t0 = tr[:, 0].min()
+        rel = (tr - t0) / 1000.0
+        phases = {name: [round(float(np.median(rel[:, i])), 2), round(float(rel[:, i].max()), 2)]
+                  for i, name in enumerate(["start", "table", "staged", "first_data", "a_done",
+                                            "b_dep", "items_done", "end"])}
+    pool.close()
+    per = expert_bytes_alg(wl)
+    alg = sum(u * per + T * wl.H * 2 + T * wl.k * wl.H * 4 for u in uniq) / len(uniq)
+    print(json.dumps({"mode": "ffn", "workload": wl.name, "layers": wl.L, "batch": T,
+                      "launch_ms_avg": round(ms, 5), "alg_bytes_per_launch": int(alg),
+                      "achieved_gbs": round(alg / (ms * 1e-3) / 1e9, 1),
+                      "phases_us_median_max": phases}), flush=True)
+
+
 # ---------------------------------------------------------------------- main
 
 def main():
@@ -225,6 +295,14 @@ def main():
     ap.add_argument("--batch", type=int, default=1, help="decode tokens per step (1, 4 or 8)")
     ap.add_argument("--all-batches", action="store_true", help="also time batches 4 and 8")
     ap.add_argument("--oracle-budget", type=float, default=10.0)
+    ap.add_argument("--mode", default="decode", choices=["decode", "ffn"],
+                    help="ffn: only the decode FFN kernel on a small all-resident pool "
+                         "(a few layers), e.g. for an ncu capture")
+    ap.add_argument("--layers", type=int, default=4, help="layer positions in --mode ffn")
+    ap.add_argument("--trace", action="store_true", help="--mode ffn: per-CTA phase timestamps")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="issue miss copies before each FFN launch (for runs under ncu, which "
+                         "serialises kernels)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -252,6 +330,9 @@ def main():
                 "wall_s": round(el, 2)}
         print(json.dumps(line), flush=True)
         return
+
+    if args.mode == "ffn":
+        return ffn_only(args, w, T)
 
     # inputs first (spawned generator workers), then CUDA
     experts = gen.expert_weights_many(w, 0, range(w.E))
@@ -285,29 +366,31 @@ def main():
                 torch.distributed.barrier()
             torch.cuda.synchronize()
             sampler.start()
-            r = decode_run(torch, m, w, pool, b, xd, wr, bias, args.steps, args.warmup, events=True)
+            r = decode_run(torch, m, w, pool, b, xd, wr, bias, args.steps, args.warmup, events=True,
+                           overlap=not args.no_overlap)
             clocks = sampler.stop()
         else:
-            r = decode_run(torch, m, w, pool, b, xd, wr, bias, args.steps, args.warmup)
+            r = decode_run(torch, m, w, pool, b, xd, wr, bias, args.steps, args.warmup,
+                           overlap=not args.no_overlap)
         res[b] = r
         del xd
 
     # e2e through the public call with host buffers
     xs_host = torch.from_numpy(np.ascontiguousarray(xs[:, :, :T]).view(np.int16)).view(torch.bfloat16).pin_memory()
-    e2e = e2e_run(torch, m, w, pool, T, xs_host, wr, bias, args.steps, args.warmup)
+    e2e = e2e_run(torch, m, w, pool, T, xs_host, wr, bias, args.steps, args.warmup,
+                  overlap=not args.no_overlap)
     pool.close()
 
     # all-resident pool: the FFN kernel's own HBM roofline on the same layers
     rpool = make_pool(m, w, w.L * w.E, 8, 1, experts)
-    xd = dev_x(T)
     preload(torch, m, rpool, w)
-    rr = decode_run(torch, m, w, rpool, T, xd, wr, bias, args.steps, args.warmup, events=True)
+    xd = dev_x(T)
+    ffn_ms, ffn_u = ffn_roofline(torch, m, w, rpool, T, xd[0], wr, bias)
     rpool.close()
-    ffn_t = [t for t, u, mm in rr["ffn"]]
-    ffn_u = [u for t, u, mm in rr["ffn"]]
     per_exp = expert_bytes_alg(w)
     alg_bytes = [u * per_exp + T * w.H * 2 + T * w.k * w.H * 4 for u in ffn_u]
-    achieved = sum(alg_bytes) / (sum(ffn_t) * 1e-3) / 1e9
+    alg_avg = sum(alg_bytes) / len(alg_bytes)
+    achieved = alg_avg / (ffn_ms * 1e-3) / 1e9
 
     # reduce over ranks: max time, summed tokens
     r = res[T]
@@ -344,8 +427,8 @@ def main():
                          "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                          "kernel": "ffn_decode_kernel", "peak_source": peak_kind,
                          "measured_on": "all-resident pool, same layers/inputs",
-                         "launch_ms_avg": round(sum(ffn_t) / len(ffn_t), 5),
-                         "alg_bytes_per_launch_avg": int(sum(alg_bytes) / len(alg_bytes))},
+                         "launch_ms_avg": round(ffn_ms, 5),
+                         "alg_bytes_per_launch_avg": int(alg_avg)},
             "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 3), "unit": "tokens/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
             "gpu_launches": 4 * w.L * args.steps,

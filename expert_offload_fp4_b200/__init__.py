@@ -6,5 +6,5 @@ is its Python binding."""
 from . import _lib  # noqa: F401
 from .api import (Lookup, Pool, combine, dequant_slot, expert_ffn, qstar_split,  # noqa: F401
                   route, route_noalloc, route_workspace_bytes, set_wait_limits, slot_lookup,
-                  stream_misses)
+                  slot_lookup_launch, slot_lookup_result, stream_misses)
 from .layer import DecodeLayer  # noqa: F401

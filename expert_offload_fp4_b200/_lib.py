@@ -64,12 +64,15 @@ SIGNATURES = {
     "moe_route_workspace_bytes": (sz, [i32, i32]),
     "moe_route": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp]),
     "moe_slot_lookup": (i32, [vp, i32, vp, i32, i32, vp, C.POINTER(LookupResult), vp]),
+    "moe_slot_lookup_launch": (i32, [vp, i32, vp, i32, i32, vp, vp]),
+    "moe_slot_lookup_result": (i32, [vp, C.POINTER(LookupResult)]),
     "moe_stream_misses": (i32, [vp, i32, C.POINTER(Miss), i32, vp]),
     "moe_expert_ffn": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp]),
     "moe_combine": (i32, [vp, i32, i32, i32, vp, vp]),
     "qstar_split": (i32, [i32, f64, f64, C.POINTER(i32), C.POINTER(i32), C.POINTER(f64)]),
     "moe_dequant_slot": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_set_wait_limits": (i32, [f64, f64, f64]),
+    "moe_set_ffn_trace": (i32, [vp]),
     "moe_route_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]),
 }
 

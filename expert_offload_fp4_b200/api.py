@@ -144,6 +144,17 @@ def slot_lookup(pool, layer, idx, slot_of, result=None, stream=None):
     return result
 
 
+def slot_lookup_launch(pool, layer, idx, slot_of, stream=None):
+    T, k = idx.shape
+    L.check("moe_slot_lookup_launch", pool.lib.moe_slot_lookup_launch(
+        pool.handle, int(layer), _p(idx), T, k, _p(slot_of), _s(stream)))
+
+
+def slot_lookup_result(pool, result):
+    L.check("moe_slot_lookup_result", pool.lib.moe_slot_lookup_result(pool.handle, C.byref(result.res)))
+    return result
+
+
 def stream_misses(pool, layer, lookup, copy_stream):
     L.check("moe_stream_misses", pool.lib.moe_stream_misses(
         pool.handle, int(layer), lookup.misses, lookup.res.n_miss, _s(copy_stream)))

@@ -52,6 +52,12 @@ struct BlockLayout {
 
 BlockLayout block_layout(const moe_config& c);
 
+// Force-load the library's kernels (lazy module loading can wait for the device,
+// which must not happen while a decode FFN waits for copies the host has yet to issue).
+int preload_router_kernels();
+int preload_lookup_kernels();
+int preload_ffn_kernels();
+
 }  // namespace moe
 
 struct moe_pool {
@@ -78,12 +84,17 @@ struct moe_pool {
     moe::LookupOut* lk_h;         // mapped pinned
     moe::LookupOut* lk_d;         // its device alias
     cudaEvent_t lk_event;
+    int lk_seq;                   // sequence number of the last launched lookup
+    int lk_pending;               // a launched lookup whose record was not collected
+    int lk_attr_set;
     // decode FFN scratch
     float* hbuf;                  // [kMaxDecodePairs][I] fp32
     unsigned int* hamax;          // [kMaxDecodePairs] |h| max as float bits
     unsigned int* ctr;            // [kMaxDecodePairs] h rows done per group, then done + abort
     // copy engine ready-flag write
     void* write_value32;          // cuStreamWriteValue32 entry point
+    int ffn_attr_set[2][5];       // decode FFN launch attributes set, per (format, token bucket)
+    int ffn_per_sm[2][5];
     moe_stats stats;
 };
 
@@ -160,6 +171,10 @@ __device__ __forceinline__ uint32_t ld_acquire_sys_u32(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+__device__ __forceinline__ void red_release_add(unsigned int* p, unsigned int v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // Named barrier over `nthreads` threads (a multiple of 32) with id `id` (1..15).

@@ -33,6 +33,7 @@ constexpr int kDoneIdx = kMaxDecodePairs + 1;
 struct Group {
     int expert, slot, M, pos;
     float ts[3];
+    float wt[kMaxDecodeT];     // routing weight of each member (token, rank)
     uint8_t tok[kMaxDecodeT];
     uint8_t rank[kMaxDecodeT];
 };
@@ -56,6 +57,7 @@ struct FfnArgs {
     int T, k, H, I, E, S, layer, fmt;
     int RA, RB, stage_bytes, nstage;
     unsigned long long ready_ns, dep_ns, pipe_ns;
+    unsigned long long* trace;   // optional [gridDim][8] phase timestamps (ns), or null
 };
 
 // ------------------------------------------------------------------ helpers
@@ -93,23 +95,66 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two) {
                        __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
 }
 
-// Power-of-two scale putting amax in [2^12, 2^13): bf16 values stay exact in f16
-// and |e2m1 * v| <= 6 * 2^13 stays finite.
+// Power-of-two scale putting amax in [2^13, 2^14): bf16 values stay exact in f16,
+// and a product with a weight (|e2m1 * 2^-14| <= 6 * 2^-14) is at most 6, so a
+// 16-product f16 block sum stays below 100.
 __device__ __forceinline__ float act_scale(float amax) {
     if (!(amax > 0.0f)) return 1.0f;
     int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-    int se = 127 + 12 - e;
+    int se = 127 + 13 - e;
     se = se < 1 ? 1 : (se > 254 ? 254 : se);
     return __uint_as_float((uint32_t)se << 23);
 }
 
-// Dot products of one row chunk (16 code bytes) against MT activation rows.
-// NVFP4: two 16-element blocks per chunk; MXFP4: one 32-element block.
+// Activations in shared memory are f16 rows stored piece-major: the 32 elements
+// of chunk c (16 code bytes) are four 16-byte pieces, piece q of chunk c at
+// uint4 index q*cpr + c (cpr = chunks per row), so lanes reading consecutive
+// chunks touch consecutive 16-byte words (no bank conflicts).  Inside a piece
+// the 8 elements are ordered 0,4,1,5,2,6,3,7: f16x2 word i holds elements
+// (i, i+4), the pairing the E2M1 decode below produces.
+__device__ __forceinline__ int act_index(int h, int cpr) {
+    const int c = h >> 5, o = h & 31, e = o & 7;
+    return (((o >> 3) * cpr + c) << 3) + (e < 4 ? 2 * e : 2 * (e - 4) + 1);
+}
+
+// 32 E2M1 codes (16 bytes; element n of a 32-bit word in bits 4n..4n+3) to 16
+// f16x2 words, each holding e2m1 * 2^-14 exactly: the code's magnitude bits go
+// to f16 bits 11..9 (exponent low bits + top mantissa bit) and its sign to bit
+// 15, so 2^-14 scales every value, the E2M1 subnormal 0.5 included.  Word 4q+i
+// holds elements (8q+i, 8q+i+4) of the chunk: one shift serves both halves.
+__device__ __forceinline__ void decode_e2m1_x2(const uint4 c, uint32_t (&w)[16]) {
+    const uint32_t v[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+        const uint32_t x = v[q];
+        w[4 * q + 0] = ((x << 9) & 0x0E000E00u) | ((x << 12) & 0x80008000u);
+        w[4 * q + 1] = ((x << 5) & 0x0E000E00u) | ((x << 8) & 0x80008000u);
+        w[4 * q + 2] = ((x << 1) & 0x0E000E00u) | ((x << 4) & 0x80008000u);
+        w[4 * q + 3] = ((x >> 3) & 0x0E000E00u) | (x & 0x80008000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ float f16x2_sum(uint32_t v) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&v);
+    const float2 f = __half22float2(h);
+    return f.x + f.y;
+}
+
+// Dot products of one row chunk (16 code bytes = 32 elements) with MT activation
+// rows.  Within a scale block the exact f16 products are summed in f16x2 (8 per
+// half for NVFP4, 16 for MXFP4); each block sum is scaled and added in fp32.
+// Weights carry 2^-14 (see decode_e2m1_x2); the caller multiplies it back.
 template <int FMT, int MT>
-__device__ __forceinline__ void chunk_dot(const uint8_t* code, const uint8_t* scl, int c,
+__device__ __forceinline__ void chunk_dot(const uint8_t* code, const uint8_t* scl, int c, int cpr,
                                           const __half* const* act, int M, float (&acc)[MT]) {
     uint32_t wv[16];
-    decode_e2m1_16B(*reinterpret_cast<const uint4*>(code + 16 * c), wv);
+    decode_e2m1_x2(*reinterpret_cast<const uint4*>(code + 16 * c), wv);
     float s0, s1;
     if (FMT == MOE_NVFP4) {
         const uint32_t two = (uint32_t)scl[2 * c] | ((uint32_t)scl[2 * c + 1] << 8);
@@ -123,20 +168,23 @@ __device__ __forceinline__ void chunk_dot(const uint8_t* code, const uint8_t* sc
 #pragma unroll
     for (int m = 0; m < MT; m++) {
         if (m >= M) break;
-        const uint4* xp = reinterpret_cast<const uint4*>(act[m] + 32 * c);
-        const uint4 x0 = xp[0], x1 = xp[1], x2 = xp[2], x3 = xp[3];
+        const uint4* xp = reinterpret_cast<const uint4*>(act[m]) + c;
+        const uint4 x0 = xp[0], x1 = xp[cpr], x2 = xp[2 * cpr], x3 = xp[3 * cpr];
         const uint32_t xv[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
                                  x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
-        float p0 = 0.0f, p1 = 0.0f;
+        uint32_t pa = 0u, pb = 0u, pc = 0u, pd = 0u;   // two chains per block
 #pragma unroll
-        for (int i = 0; i < 8; i++) p0 = fma_f16x2(wv[i], xv[i], p0);
-#pragma unroll
-        for (int i = 8; i < 16; i++) p1 = fma_f16x2(wv[i], xv[i], p1);
+        for (int i = 0; i < 8; i += 2) {
+            pa = hfma2_u32(wv[i], xv[i], pa);
+            pb = hfma2_u32(wv[i + 1], xv[i + 1], pb);
+            pc = hfma2_u32(wv[8 + i], xv[8 + i], pc);
+            pd = hfma2_u32(wv[9 + i], xv[9 + i], pd);
+        }
         if (FMT == MOE_NVFP4) {
-            acc[m] = fmaf(p0, s0, acc[m]);
-            acc[m] = fmaf(p1, s1, acc[m]);
+            acc[m] = fmaf(f16x2_sum(pa) + f16x2_sum(pb), s0, acc[m]);
+            acc[m] = fmaf(f16x2_sum(pc) + f16x2_sum(pd), s1, acc[m]);
         } else {
-            acc[m] = fmaf(p0 + p1, s0, acc[m]);
+            acc[m] = fmaf((f16x2_sum(pa) + f16x2_sum(pb)) + (f16x2_sum(pc) + f16x2_sum(pd)), s0, acc[m]);
         }
     }
 }
@@ -176,7 +224,7 @@ __device__ __forceinline__ bool wait_ready(const FfnArgs& a, int slot, volatile 
         if (ld_acquire_sys_u32(a.ready + slot) == want) return true;
         if (*abort_flag) return false;
         if (globaltimer() - t0 > a.ready_ns) return false;
-        __nanosleep(200);
+        __nanosleep(64);
     }
 }
 
@@ -197,77 +245,146 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     volatile unsigned int* abort_flag = a.ctr + kAbortIdx;
+    unsigned long long* trace = a.trace ? a.trace + (size_t)blockIdx.x * 8 : nullptr;
+    if (trace && tid == 0) trace[0] = globaltimer();
     const int bs = FMT == MOE_MXFP4 ? 32 : 16;
     const unsigned long long codeA = (unsigned long long)a.H / 2, sclA = (unsigned long long)a.H / bs;
     const unsigned long long codeB = (unsigned long long)a.I / 2, sclB = (unsigned long long)a.I / bs;
 
-    // ---- prologue: barriers, groups, activations
+    // ---- prologue: barriers, groups, activations (parallel; the stage ring is
+    // still unused, so its first bytes hold the per-(token, rank) scratch)
+    int* e_s = reinterpret_cast<int*>(stages);            // [n] expert or -1
+    int* s_s = e_s + kMaxDecodePairs;                      // [n] slot
+    unsigned* need_s = reinterpret_cast<unsigned*>(s_s + kMaxDecodePairs);
+    int* lead_s = reinterpret_cast<int*>(need_s + kMaxDecodePairs);   // first entry of my expert
+    int* mi_s = lead_s + kMaxDecodePairs;                  // my index inside the group
+    int* grank_s = mi_s + kMaxDecodePairs;                 // group rank of a leader
+    const int n = a.T * a.k;
     if (tid == 0) {
         for (int i = 0; i < a.nstage; i++) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kNC);
         }
         fence_mbar_init();
-        int ng = 0, bad = 0;
-        const int n = a.T * a.k;
-        for (int i = 0; i < n; i++) {
-            const int e = a.idx[i], s = a.slot_of[i];
-            if (e < 0 || e >= a.E) { bad |= MOE_STATUS_BAD_EXPERT; continue; }
-            if (s < 0 || s >= a.S) { bad |= MOE_STATUS_BAD_SLOT; continue; }
-            int g = 0;
-            while (g < ng && groups[g].expert != e) g++;
-            if (g == ng) {
-                groups[g].expert = e;
-                groups[g].slot = s;
-                groups[g].M = 0;
-                const float* ts = a.tscale + ((size_t)a.layer * a.E + e) * 3;
-                groups[g].ts[0] = ts[0];
-                groups[g].ts[1] = ts[1];
-                groups[g].ts[2] = ts[2];
-                ng++;
-            }
-            Group& G = groups[g];
-            G.tok[G.M] = (uint8_t)(i / a.k);
-            G.rank[G.M] = (uint8_t)(i % a.k);
-            G.M++;
-        }
-        // ascending ticket the slot must show: resident experts first, misses in copy order
-        for (int i = 1; i < ng; i++) {
-            Group key = groups[i];
-            const uint32_t kt = a.need[key.slot];
-            int j = i - 1;
-            while (j >= 0 && (a.need[groups[j].slot] > kt ||
-                              (a.need[groups[j].slot] == kt && groups[j].expert > key.expert))) {
-                groups[j + 1] = groups[j];
-                j--;
-            }
-            groups[j + 1] = key;
-        }
-        int pos = 0;
-        for (int g = 0; g < ng; g++) {
-            groups[g].pos = pos;
-            pos += groups[g].M;
-        }
-        s_misc[0] = ng;
+    }
+    if (tid < n) {
+        const int e = a.idx[tid], sl = a.slot_of[tid];
+        int bad = 0;
+        if (e < 0 || e >= a.E) bad |= MOE_STATUS_BAD_EXPERT;
+        if (sl < 0 || sl >= a.S) bad |= MOE_STATUS_BAD_SLOT;
+        e_s[tid] = bad ? -1 : e;
+        s_s[tid] = sl;
+        need_s[tid] = bad ? 0u : a.need[sl];
         if (bad && blockIdx.x == 0) atomicOr(a.status, bad);
     }
-    // activations: per-token power-of-two scale, f16
-    for (int t = warp; t < a.T; t += kNC + 1) {
-        float amax = 0.0f;
-        for (int h = lane; h < a.H; h += 32)
-            amax = fmaxf(amax, fabsf(__uint_as_float((uint32_t)a.x[(size_t)t * a.H + h] << 16)));
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        const float sc = act_scale(amax);
-        if (lane == 0) xinv[t] = 1.0f / sc;
-        for (int h = lane; h < a.H; h += 32)
-            xs[t * a.H + h] = __float2half_rn(__uint_as_float((uint32_t)a.x[(size_t)t * a.H + h] << 16) * sc);
+    __syncthreads();
+    if (tid < n && e_s[tid] >= 0) {
+        const int e = e_s[tid];
+        int lead = tid, mi = 0;
+        for (int j = 0; j < tid; j++)
+            if (e_s[j] == e) {
+                if (lead == tid) lead = j;
+                mi++;
+            }
+        lead_s[tid] = lead;
+        mi_s[tid] = mi;
     }
     __syncthreads();
-
+    // leaders: rank by (ticket the slot must show, expert) so resident experts come
+    // first and missed ones in the order the copy engine delivers them
+    if (tid < n && e_s[tid] >= 0 && lead_s[tid] == tid) {
+        const int e = e_s[tid];
+        const unsigned kt = need_s[tid];
+        int rank = 0, M = 0, pos = 0;
+        for (int j = 0; j < n; j++) {
+            const int ej = e_s[j];
+            if (ej < 0) continue;
+            if (ej == e) M++;
+            const bool before = need_s[j] < kt || (need_s[j] == kt && ej < e);
+            if (lead_s[j] == j && before) rank++;
+            if (before) pos++;       // members of groups ranked before mine
+        }
+        grank_s[tid] = rank;
+        Group& G = groups[rank];
+        G.expert = e;
+        G.slot = s_s[tid];
+        G.M = M;
+        G.pos = pos;
+        const float* ts = a.tscale + ((size_t)a.layer * a.E + e) * 3;
+        G.ts[0] = ts[0];
+        G.ts[1] = ts[1];
+        G.ts[2] = ts[2];
+    }
+    __syncthreads();
+    if (tid < n && e_s[tid] >= 0) {
+        Group& G = groups[grank_s[lead_s[tid]]];
+        G.tok[mi_s[tid]] = (uint8_t)(tid / a.k);
+        G.rank[mi_s[tid]] = (uint8_t)(tid % a.k);
+        G.wt[mi_s[tid]] = a.w[tid];
+    }
+    if (warp == 0) {
+        int c = 0;
+        for (int i = lane; i < n; i += 32) c += (e_s[i] >= 0 && lead_s[i] == i);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+        if (lane == 0) s_misc[0] = c;
+    }
+    __syncthreads();
+    // from here the producer warp streams weights while the consumers stage the
+    // activations: per-token power-of-two scale, f16, piece-major rows, 16-byte
+    // loads (8 bf16), a shared per-token max first (in hinv, free until the
+    // down projection)
+    const int cprA = a.H / 32, cprB = a.I / 32;
+    if (warp < kNC) {
+        unsigned* tok_amax = reinterpret_cast<unsigned*>(hinv);
+        if (tid < a.T) tok_amax[tid] = 0u;
+        named_sync(2, kNC * 32);
+        const int nvec = a.T * a.H / 8;
+        for (int v = tid; v < nvec; v += kNC * 32) {
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(a.x) + v);
+            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+            float mx = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(u[i] << 16)), fabsf(__uint_as_float(u[i] & 0xFFFF0000u))));
+            atomicMax(tok_amax + (v * 8) / a.H, __float_as_uint(mx));
+        }
+        named_sync(2, kNC * 32);
+        for (int v = tid; v < nvec; v += kNC * 32) {
+            const int t = (v * 8) / a.H, h = v * 8 - t * a.H;
+            const float sc = act_scale(__uint_as_float(tok_amax[t]));
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(a.x) + v);
+            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                f[2 * i] = __uint_as_float(u[i] << 16) * sc;
+                f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u) * sc;
+            }
+            // one piece: f16x2 words (0,4), (1,5), (2,6), (3,7)
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const __half2 h2 = __floats2half2_rn(f[i], f[i + 4]);
+                o[i] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            *reinterpret_cast<uint4*>(xs + t * a.H + act_index(h, cprA)) = make_uint4(o[0], o[1], o[2], o[3]);
+            if (h == 0) xinv[t] = 1.0f / sc;
+        }
+        named_sync(2, kNC * 32);
+    }
+    if (trace && tid == 0) trace[2] = globaltimer();
     const int ng = s_misc[0];
     const int nA_per = a.I / a.RA, nB_per = a.H / a.RB;
-    const int NA = ng * nA_per, N = NA + ng * nB_per;
+    const int NA = ng * nA_per, NB = ng * nB_per;
+    // contiguous item ranges per CTA (consecutive items mostly share an expert):
+    // this CTA's A items, then its B items
+    const int a0 = (int)((long long)blockIdx.x * NA / gridDim.x);
+    const int a1 = (int)((long long)(blockIdx.x + 1) * NA / gridDim.x);
+    const int b0 = (int)((long long)blockIdx.x * NB / gridDim.x);
+    const int b1 = (int)((long long)(blockIdx.x + 1) * NB / gridDim.x);
+    const int nmine = (a1 - a0) + (b1 - b0);
+    auto item_of = [&](int j) { return j < a1 - a0 ? a0 + j : NA + b0 + (j - (a1 - a0)); };
 
     auto stage_map = [&](int item, unsigned long long* src, uint32_t* len, int& nsrc) -> StageMap {
         StageMap m{};
@@ -318,19 +435,37 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
     if (warp == kNC) {
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
-            int it = 0;
-            for (int item = blockIdx.x; item < N; item += gridDim.x, it++) {
-                const int st = it % a.nstage, round = it / a.nstage;
+            // one sweep over the groups this CTA touches: experts already resident
+            // (or landed) are marked ready behind a single proxy fence; the others are
+            // waited for when their first item comes up
+            uint32_t ready_mask[kMaxDecodePairs / 32] = {0, 0, 0, 0};
+            int any = 0;
+            for (int j = 0; j < nmine; j++) {
+                const int item = item_of(j);
+                const int g = item >= NA ? (item - NA) / nB_per : item / nA_per;
+                if (ready_mask[g >> 5] & (1u << (g & 31))) continue;
+                if (ld_acquire_u32(a.ready + groups[g].slot) == a.need[groups[g].slot]) {
+                    ready_mask[g >> 5] |= 1u << (g & 31);
+                    any = 1;
+                }
+            }
+            if (any) fence_proxy_async_global();
+            for (int j = 0; j < nmine; j++) {
+                const int item = item_of(j);
+                const int st = j % a.nstage, round = j / a.nstage;
                 if (!mbar_wait(&empty[st], (round & 1) ^ 1, a.pipe_ns)) {
                     atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
                     *abort_flag = 1;
                 }
                 const int g = item >= NA ? (item - NA) / nB_per : item / nA_per;
-                if (!wait_ready(a, groups[g].slot, abort_flag)) {
-                    atomicOr(a.status, MOE_STATUS_READY_TIMEOUT);
-                    *abort_flag = 1;
+                if (!(ready_mask[g >> 5] & (1u << (g & 31)))) {
+                    if (!wait_ready(a, groups[g].slot, abort_flag)) {
+                        atomicOr(a.status, MOE_STATUS_READY_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    ready_mask[g >> 5] |= 1u << (g & 31);
+                    fence_proxy_async_global();
                 }
-                fence_proxy_async_global();
                 unsigned long long src[4];
                 uint32_t len[4];
                 int nsrc = 0;
@@ -345,21 +480,32 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
             }
             // no copy may still be in flight when the CTA exits: wait (bounded) for
             // the last phase of every stage used
-            for (int j = (it > a.nstage ? it - a.nstage : 0); j < it; j++)
+            for (int j = (nmine > a.nstage ? nmine - a.nstage : 0); j < nmine; j++)
                 if (!mbar_wait(&full[j % a.nstage], (j / a.nstage) & 1, a.pipe_ns))
                     atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
         }
     } else {
         // ---------------------------------------------------------------- consumers
         const int GA = lanes_per_row(a.H), GB = lanes_per_row(a.I);
-        int it = 0;
-        for (int item = blockIdx.x; item < N; item += gridDim.x, it++) {
-            const int st = it % a.nstage, round = it / a.nstage;
+        int pend_g = -1, pend_n = 0;   // h rows written by this warp, not yet published
+        auto publish = [&]() {
+            __syncwarp();
+            if (lane == 0 && pend_n > 0) {
+                __threadfence();
+                atomicAdd(a.ctr + pend_g, (unsigned int)pend_n);
+            }
+            pend_n = 0;
+        };
+        int staged_g = -1;             // group whose h sits in hs (same on every consumer warp)
+        for (int j = 0; j < nmine; j++) {
+            const int item = item_of(j);
+            const int st = j % a.nstage, round = j / a.nstage;
             const bool ok = mbar_wait(&full[st], round & 1, a.pipe_ns);
             if (!ok) {
                 if (lane == 0) atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
                 *abort_flag = 1;
             }
+            if (trace && tid == 0 && j == 0) trace[3] = globaltimer();
             unsigned long long src[4];
             uint32_t len[4];
             int nsrc;
@@ -371,12 +517,15 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
             const int M = G.M;
             if (!isB) {
                 // A: gate row p and up row p of this item per lane group
+                if (g != pend_g) {
+                    publish();
+                    pend_g = g;
+                }
                 const int rb = item % nA_per;
                 const int RW = 32 / GA, sub = lane / GA, gl = lane % GA;
                 const __half* act[MT];
 #pragma unroll
                 for (int q = 0; q < MT; q++) act[q] = xs + (size_t)G.tok[q < M ? q : 0] * a.H;
-                int rows_done = 0;
                 for (int base = 0; base < a.RA; base += kNC * RW) {
                     const int p = base + warp * RW + sub;
                     float ag[MT], au[MT];
@@ -387,9 +536,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                         const uint8_t* gs = sb + m.scl0 + m.scl0_in + (size_t)p * sclA;
                         const uint8_t* uc = sb + m.codes1 + (size_t)p * codeA;
                         const uint8_t* us = sb + m.scl1 + m.scl1_in + (size_t)p * sclA;
-                        for (int c = gl; c < (int)(codeA / 16); c += GA) {
-                            chunk_dot<FMT, MT>(gc, gs, c, act, M, ag);
-                            chunk_dot<FMT, MT>(uc, us, c, act, M, au);
+#pragma unroll 2
+                        for (int c = gl; c < cprA; c += GA) {
+                            chunk_dot<FMT, MT>(gc, gs, c, cprA, act, M, ag);
+                            chunk_dot<FMT, MT>(uc, us, c, cprA, act, M, au);
                         }
                     }
                     group_reduce<MT>(ag, GA);
@@ -399,52 +549,62 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
 #pragma unroll
                         for (int q = 0; q < MT; q++) {
                             if (q >= M) break;
-                            const float xi = xinv[G.tok[q]];
+                            const float xi = xinv[G.tok[q]] * 16384.0f;   // undo the decode's 2^-14
                             const float gv = ag[q] * xi * G.ts[0];
                             const float uv = au[q] * xi * G.ts[1];
                             const float hv = gv / (1.0f + expf(-gv)) * uv;
                             a.hbuf[(size_t)(G.pos + q) * a.I + i] = hv;
                             atomicMax(a.hamax + G.pos + q, __float_as_uint(fabsf(hv)));
                         }
-                        rows_done++;
                     }
+                    // rows this warp finished in this pass (the same count on every lane)
+                    const int left = a.RA - (base + warp * RW);
+                    pend_n += left <= 0 ? 0 : (left < RW ? left : RW);
                 }
-                // publish: every writer fences, the warp syncs, lane 0 bumps the counter
-                __threadfence();
-                __syncwarp();
-#pragma unroll
-                for (int off = 16; off >= 1; off >>= 1) rows_done += __shfl_xor_sync(0xffffffffu, rows_done, off);
-                if (lane == 0 && rows_done) {
-                    __threadfence();
-                    atomicAdd(a.ctr + g, (unsigned int)rows_done);
+                if (j + 1 == a1 - a0) {             // last A item of this CTA
+                    publish();
+                    if (trace && tid == 0) trace[4] = globaltimer();
                 }
             } else {
-                // B: wait for all I rows of h, stage it in f16, then RB rows of down
-                const int rb = (item - NA) % nB_per;
-                if (warp == 0 && lane == 0) {
-                    const unsigned int want = (unsigned int)a.I;
-                    if (ld_acquire_u32(a.ctr + g) < want) {
-                        const unsigned long long t0 = globaltimer();
-                        while (ld_acquire_u32(a.ctr + g) < want) {
-                            if (*abort_flag || globaltimer() - t0 > a.dep_ns) {
-                                atomicOr(a.status, MOE_STATUS_DEP_TIMEOUT);
-                                *abort_flag = 1;
-                                break;
+                // B: h of the group staged once per run of its items, then RB rows of down
+                if (g != staged_g) {
+                    if (warp == 0 && lane == 0) {
+                        const unsigned int want = (unsigned int)a.I;
+                        if (ld_acquire_u32(a.ctr + g) < want) {
+                            const unsigned long long t0 = globaltimer();
+                            while (ld_acquire_u32(a.ctr + g) < want) {
+                                if (*abort_flag || globaltimer() - t0 > a.dep_ns) {
+                                    atomicOr(a.status, MOE_STATUS_DEP_TIMEOUT);
+                                    *abort_flag = 1;
+                                    break;
+                                }
                             }
-                            __nanosleep(100);
                         }
                     }
+                    if (trace && tid == 0 && staged_g < 0) trace[5] = globaltimer();
+                    named_sync(1, kNC * 32);   // also: every warp is done with the old hs
+                    for (int q = warp; q < M; q += kNC) {
+                        const float amax = __uint_as_float(__ldcg(a.hamax + G.pos + q));
+                        const float sc = act_scale(amax);
+                        if (lane == 0) hinv[q] = 1.0f / sc;
+                        const float4* hrow = reinterpret_cast<const float4*>(a.hbuf + (size_t)(G.pos + q) * a.I);
+                        for (int v = lane; v < a.I / 8; v += 32) {
+                            const float4 f0 = __ldcg(hrow + 2 * v), f1 = __ldcg(hrow + 2 * v + 1);
+                            const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                            uint32_t o[4];
+#pragma unroll
+                            for (int i = 0; i < 4; i++) {
+                                const __half2 h2 = __floats2half2_rn(f[i] * sc, f[i + 4] * sc);
+                                o[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                            }
+                            *reinterpret_cast<uint4*>(hs + (size_t)q * a.I + act_index(8 * v, cprB)) =
+                                make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                    named_sync(1, kNC * 32);
+                    staged_g = g;
                 }
-                named_sync(1, kNC * 32);
-                __threadfence();
-                for (int q = warp; q < M; q += kNC) {
-                    const float amax = __uint_as_float(__ldcg(a.hamax + G.pos + q));
-                    const float sc = act_scale(amax);
-                    if (lane == 0) hinv[q] = 1.0f / sc;
-                    const float* hrow = a.hbuf + (size_t)(G.pos + q) * a.I;
-                    for (int i = lane; i < a.I; i += 32) hs[q * a.I + i] = __float2half_rn(__ldcg(hrow + i) * sc);
-                }
-                named_sync(1, kNC * 32);
+                const int rb = (item - NA) % nB_per;
                 const int RW = 32 / GB, sub = lane / GB, gl = lane % GB;
                 const __half* act[MT];
 #pragma unroll
@@ -457,7 +617,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                     if (r < a.RB && ok) {
                         const uint8_t* dc = sb + m.codes0 + (size_t)r * codeB;
                         const uint8_t* ds = sb + m.scl0 + m.scl0_in + (size_t)r * sclB;
-                        for (int c = gl; c < (int)(codeB / 16); c += GB) chunk_dot<FMT, MT>(dc, ds, c, act, M, ay);
+#pragma unroll 2
+                        for (int c = gl; c < cprB; c += GB) chunk_dot<FMT, MT>(dc, ds, c, cprB, act, M, ay);
                     }
                     group_reduce<MT>(ay, GB);
                     if (r < a.RB && gl == 0) {
@@ -465,21 +626,23 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
 #pragma unroll
                         for (int q = 0; q < MT; q++) {
                             if (q >= M) break;
-                            const int t = G.tok[q], j = G.rank[q];
-                            const float wt = a.w[t * a.k + j];
-                            a.y_part[((size_t)t * a.k + j) * a.H + row] = wt * (ay[q] * hinv[q] * G.ts[2]);
+                            const int t = G.tok[q], jr = G.rank[q];
+                            a.y_part[((size_t)t * a.k + jr) * a.H + row] =
+                                G.wt[q] * (ay[q] * (hinv[q] * 16384.0f) * G.ts[2]);
                         }
                     }
                 }
-                named_sync(1, kNC * 32);  // hs is rewritten by the next B item
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
+        publish();
+        if (trace && tid == 0) trace[6] = globaltimer();
     }
 
     // ---- epilogue: the last CTA clears the per-call counters
     __syncthreads();
+    if (trace && tid == 0) trace[7] = globaltimer();
     if (tid == 0) {
         __threadfence();
         const unsigned int prev = atomicAdd(a.ctr + kDoneIdx, 1u);
@@ -577,9 +740,17 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     const size_t smem = 16 * (size_t)a.nstage + sizeof(Group) * kMaxDecodePairs + 4 * (2 * kMaxDecodeT + 4) + 16 +
                         (size_t)a.T * c.H * 2 + (size_t)MT * c.I * 2 + 128 + (size_t)a.nstage * a.stage_bytes;
     auto kern = ffn_decode_kernel<FMT, MT>;
-    MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    int per_sm = 0;
-    MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFfnThreads, smem));
+    const int fi = FMT == MOE_NVFP4 ? 1 : 0, mi = MT == 1 ? 0 : MT == 2 ? 1 : MT == 4 ? 2 : MT == 8 ? 3 : 4;
+    if (!p->ffn_attr_set[fi][mi]) {
+        // once per pool and template: the largest shared-memory carve-out, and the
+        // number of co-resident CTAs per SM at that size (1: the kernel is persistent)
+        MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget));
+        int per_sm = 0;
+        MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFfnThreads, budget));
+        p->ffn_per_sm[fi][mi] = per_sm;
+        p->ffn_attr_set[fi][mi] = 1;
+    }
+    const int per_sm = p->ffn_per_sm[fi][mi];
     if (per_sm < 1) return fail(MOE_EINVAL, "decode FFN kernel does not fit on an SM");
     const int items_max = a.T * a.k * (c.I / a.RA + c.H / a.RB);
     const int grid = std::max(1, std::min(p->num_sms * per_sm, items_max));
@@ -588,11 +759,33 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     return MOE_OK;
 }
 
+int preload_ffn_kernels() {
+    cudaFuncAttributes fa;
+#define PRELOAD(F)                                                           \
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, ffn_decode_kernel<F, 1>));       \
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, ffn_decode_kernel<F, 2>));       \
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, ffn_decode_kernel<F, 4>));       \
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, ffn_decode_kernel<F, 8>));       \
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, ffn_decode_kernel<F, 16>));      \
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, dequant_kernel<F>));
+    PRELOAD(MOE_NVFP4)
+    PRELOAD(MOE_MXFP4)
+#undef PRELOAD
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, combine_kernel));
+    return MOE_OK;
+}
+
 }  // namespace moe
 
 using namespace moe;
 
 static unsigned long long g_ready_ns = 5000000000ull, g_dep_ns = 5000000000ull, g_pipe_ns = 10000000000ull;
+static unsigned long long* g_trace = nullptr;
+
+extern "C" int moe_set_ffn_trace(void* buf) {
+    g_trace = (unsigned long long*)buf;
+    return MOE_OK;
+}
 
 extern "C" int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms) {
     if (!(ready_ms > 0) || !(dep_ms > 0) || !(pipe_ms > 0)) return fail(MOE_EINVAL, "wait limits must be positive");
@@ -636,6 +829,7 @@ extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T,
     a.ready_ns = g_ready_ns;
     a.dep_ns = g_dep_ns;
     a.pipe_ns = g_pipe_ns;
+    a.trace = g_trace;
     cudaStream_t s = (cudaStream_t)stream;
     const int MT = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16;
 #define DISPATCH(F)                                              \

@@ -241,23 +241,27 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(LookupArgs a) {
     }
 }
 
+int preload_lookup_kernels() {
+    cudaFuncAttributes fa;
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, lookup_kernel));
+    return MOE_OK;
+}
+
 }  // namespace moe
 
 using namespace moe;
 
-extern "C" int moe_slot_lookup(moe_pool* p, int layer, const int32_t* idx, int T, int k,
-                               int32_t* slot_of, moe_lookup_result* res, void* stream) {
-    if (!p || !idx || !slot_of || !res) return fail(MOE_EINVAL, "null argument");
+extern "C" int moe_slot_lookup_launch(moe_pool* p, int layer, const int32_t* idx, int T, int k,
+                                      int32_t* slot_of, void* stream) {
+    if (!p || !idx || !slot_of) return fail(MOE_EINVAL, "null argument");
     const moe_config& c = p->cfg;
     if (layer < 0 || layer >= c.L) return fail(MOE_EBOUNDS, "layer outside the pool");
     if (T <= 0 || k <= 0 || k > c.E || (long long)T * k > (1LL << 24)) return fail(MOE_EINVAL, "bad T/k");
     // the pool must hold every expert one call can touch, or a miss finds no victim
     const int cap = T * k < c.E ? T * k : c.E;
     if (cap > c.n_slots) return fail(MOE_EINVAL, "slot pool smaller than the unique experts one call can touch");
-    if (!res->uniq_h || !res->is_hit_h || !res->miss_h) return fail(MOE_EINVAL, "null result arrays");
+    if (p->lk_pending) return fail(MOE_ESTATE, "a launched lookup has not been collected");
     cudaStream_t s = (cudaStream_t)stream;
-    static thread_local int seq = 0;
-    seq++;
     LookupArgs a;
     a.idx = idx;
     a.n = T * k;
@@ -272,24 +276,39 @@ extern "C" int moe_slot_lookup(moe_pool* p, int layer, const int32_t* idx, int T
     a.need = p->need;
     a.slot_of = slot_of;
     a.out = p->lk_d;
-    a.seq = seq;
+    a.seq = ++p->lk_seq;
     const size_t smem = size_t(2) * ((c.n_slots + 31) / 32) * sizeof(uint32_t);
     if (smem > 160 * 1024) return fail(MOE_EINVAL, "n_slots too large for the lookup kernel");
-    MOE_CUDA_TRY(cudaFuncSetAttribute(lookup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    if (!p->lk_attr_set) {
+        MOE_CUDA_TRY(cudaFuncSetAttribute(lookup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+        p->lk_attr_set = 1;
+    }
     lookup_kernel<<<1, kLookupThreads, smem, s>>>(a);
     MOE_CUDA_TRY(cudaGetLastError());
     MOE_CUDA_TRY(cudaEventRecord(p->lk_event, s));
+    p->lk_pending = 1;
+    return MOE_OK;
+}
+
+extern "C" int moe_slot_lookup_result(moe_pool* p, moe_lookup_result* res) {
+    if (!p || !res) return fail(MOE_EINVAL, "null argument");
+    if (!res->uniq_h || !res->is_hit_h || !res->miss_h) return fail(MOE_EINVAL, "null result arrays");
+    if (!p->lk_pending) return fail(MOE_ESTATE, "no launched lookup to collect");
     // bounded host wait: the copy engine can only be driven once the miss list is known
     const auto t0 = std::chrono::steady_clock::now();
     while (true) {
         cudaError_t q = cudaEventQuery(p->lk_event);
         if (q == cudaSuccess) break;
-        if (q != cudaErrorNotReady) return cuda_fail(q, "lookup kernel");
+        if (q != cudaErrorNotReady) {
+            p->lk_pending = 0;
+            return cuda_fail(q, "lookup kernel");
+        }
         if (std::chrono::steady_clock::now() - t0 > std::chrono::seconds(10))
             return fail(MOE_ETIMEOUT, "lookup kernel did not finish within 10 s");
     }
+    p->lk_pending = 0;
     volatile LookupOut* o = p->lk_h;
-    if (o->seq != seq) return fail(MOE_ECUDA, "lookup record not written");
+    if (o->seq != p->lk_seq) return fail(MOE_ECUDA, "lookup record not written");
     if (o->status) return fail(MOE_EBOUNDS, "expert index outside [0, E)");
     res->n_uniq = o->n_uniq;
     res->n_miss = o->n_miss;
@@ -311,4 +330,13 @@ extern "C" int moe_slot_lookup(moe_pool* p, int layer, const int32_t* idx, int T
     p->stats.hits += o->n_uniq - o->n_miss;
     for (int r = 0; r < o->n_miss; r++) p->stats.evictions += o->miss[r].evicted_key >= 0;
     return MOE_OK;
+}
+
+extern "C" int moe_slot_lookup(moe_pool* p, int layer, const int32_t* idx, int T, int k,
+                               int32_t* slot_of, moe_lookup_result* res, void* stream) {
+    if (!res) return fail(MOE_EINVAL, "null argument");
+    if (!res->uniq_h || !res->is_hit_h || !res->miss_h) return fail(MOE_EINVAL, "null result arrays");
+    int rc = moe_slot_lookup_launch(p, layer, idx, T, k, slot_of, stream);
+    if (rc) return rc;
+    return moe_slot_lookup_result(p, res);
 }

@@ -165,6 +165,10 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
         moe_pool_destroy(p);
         return rc;
     }
+    if ((rc = preload_router_kernels()) || (rc = preload_lookup_kernels()) || (rc = preload_ffn_kernels())) {
+        moe_pool_destroy(p);
+        return rc;
+    }
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) { rc = cuda_fail(e, "pool init"); moe_pool_destroy(p); return rc; }
     *out = p;

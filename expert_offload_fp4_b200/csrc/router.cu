@@ -155,8 +155,15 @@ static cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const fl
                                  float* logits, unsigned int* cnt, cudaStream_t s) {
     const size_t smem = size_t(TT) * H * sizeof(float);
     auto kern = router_kernel<EPW, TT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    // the x tile is at most 200 KiB (checked by the caller); raise the limit once per device
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = true;
+    }
     dim3 grid((E + kRouterWarps * EPW - 1) / (kRouterWarps * EPW), (T + TT - 1) / TT);
     kern<<<grid, kRouterWarps * 32, smem, s>>>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt);
     return cudaGetLastError();
@@ -180,6 +187,17 @@ int route_impl(const void* x_bf16, const void* wr_bf16, const float* bias, int T
     else if (T <= 8) e = launch_router<2, 8>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt, s);
     else e = launch_router<4, 8>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt, s);
     if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    return MOE_OK;
+}
+
+// Load every router instantiation now (module loading may wait for the device).
+int preload_router_kernels() {
+    cudaFuncAttributes fa;
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, router_kernel<1, 1>));
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, router_kernel<1, 2>));
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, router_kernel<1, 4>));
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, router_kernel<2, 8>));
+    MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, router_kernel<4, 8>));
     return MOE_OK;
 }
 

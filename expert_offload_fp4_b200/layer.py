@@ -14,10 +14,12 @@ from . import api
 
 
 class DecodeLayer:
-    def __init__(self, pool: api.Pool, T: int, device="cuda", renormalize=1):
+    def __init__(self, pool: api.Pool, T: int, device="cuda", renormalize=1, overlap=True):
         if T > pool.max_tokens:
             raise ValueError("T exceeds the pool's max_tokens")
-        self.pool, self.T, self.renormalize = pool, T, renormalize
+        # overlap=False issues the miss copies before the FFN launch (the host waits
+        # for the lookup first): slower, but safe under tools that serialise kernels
+        self.pool, self.T, self.renormalize, self.overlap = pool, T, renormalize, overlap
         k, H, E = pool.k, pool.H, pool.E
         self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
         self.w = torch.empty((T, k), dtype=torch.float32, device=device)
@@ -35,10 +37,32 @@ class DecodeLayer:
 
     def __call__(self, layer, x, wr, bias, stream=None):
         """x [T, H] bf16, wr [E, H] bf16, bias [E] fp32 (or None), all on the device.
-        Returns y [T, H] bf16 (a buffer reused by the next call)."""
+        Returns y [T, H] bf16 (a buffer reused by the next call).
+
+        Order: route, lookup, FFN and combine are enqueued back to back on the
+        compute stream; then the host collects the lookup's miss list and drives
+        the copy engine.  The FFN's CTAs on resident experts run at once; those on
+        missed experts wait (bounded) for the slot's ready ticket that the copy
+        stream writes after each expert's block lands."""
         p = self.pool
         api.route(x, wr, bias, p.k, self.renormalize, self.idx, self.w, self.ws, stream)
-        api.slot_lookup(p, layer, self.idx, self.slot_of, self.lookup, stream)
+        if not self.overlap:
+            api.slot_lookup(p, layer, self.idx, self.slot_of, self.lookup, stream)
+            if self.lookup.n_miss:
+                api.stream_misses(p, layer, self.lookup, self.copy_stream)
+            api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, stream)
+            api.combine(self.y_part, self.y, stream)
+            return self.y
+        api.slot_lookup_launch(p, layer, self.idx, self.slot_of, stream)
+        if self.ffn_events is not None:
+            cur = stream if stream is not None else torch.cuda.current_stream()
+            fe = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            fe[0].record(cur)
+        api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, stream)
+        if self.ffn_events is not None:
+            fe[1].record(cur)
+        # nothing that can wait for the device between the FFN launch and the copies
+        api.slot_lookup_result(p, self.lookup)
         if self.lookup.n_miss:
             if self.copy_events is not None:
                 ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -47,13 +71,7 @@ class DecodeLayer:
             if self.copy_events is not None:
                 ev[1].record(self.copy_stream)
                 self.copy_events.append((ev, self.lookup.n_miss))
-        if self.ffn_events is not None:
-            cur = stream if stream is not None else torch.cuda.current_stream()
-            fe = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            fe[0].record(cur)
-        api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, stream)
-        if self.ffn_events is not None:
-            fe[1].record(cur)
-            self.ffn_events.append((fe, self.lookup.n_uniq, self.lookup.n_miss))
         api.combine(self.y_part, self.y, stream)
+        if self.ffn_events is not None:
+            self.ffn_events.append((fe, self.lookup.n_uniq, self.lookup.n_miss))
         return self.y

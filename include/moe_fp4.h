@@ -179,13 +179,27 @@ int moe_route_noalloc(const void* x_bf16, const void* wr_bf16, const float* bias
 int moe_slot_lookup(moe_pool* pool, int layer, const int32_t* idx, int T, int k, int32_t* slot_of,
                     moe_lookup_result* res, void* stream);
 
+/* The two halves of moe_slot_lookup, so that the FFN of the same layer can be
+ * enqueued before the host learns the misses: _launch enqueues the lookup kernel
+ * (slot_of and the slot tickets are then final in stream order); _result waits
+ * (bounded, MOE_ETIMEOUT after 10 s) for it and fills *res.  One lookup may be
+ * outstanding per pool (MOE_ESTATE otherwise). */
+int moe_slot_lookup_launch(moe_pool* pool, int layer, const int32_t* idx, int T, int k,
+                           int32_t* slot_of, void* stream);
+int moe_slot_lookup_result(moe_pool* pool, moe_lookup_result* res);
+
 /* Miss streaming ("游戏电脑如何跑动2840亿参数大模型": prefetch with a double
  * buffer, copies in the background while computing).  For each miss, in order,
  * one cudaMemcpyAsync of the expert's pinned host block into its slot on
  * copy_stream, then a stream write of the ticket into the slot's ready flag.
  * moe_expert_ffn starts at once on another stream; its CTAs on missed experts
  * wait (bounded) for the flag, so the copy of miss j+1 overlaps compute on the
- * hits and on miss j.  Errors: MOE_EBOUNDS, MOE_ESTATE (expert never loaded). */
+ * hits and on miss j.  When the FFN is enqueued before the misses are streamed
+ * (moe_slot_lookup_launch, moe_expert_ffn, moe_slot_lookup_result, then this
+ * call), the host must not wait for the device in between (a synchronize, a
+ * blocking allocation, a first launch of a lazily loaded kernel): the FFN would
+ * wait for copies not yet issued until its bounded wait gives up.  The pool
+ * loads all of the library's kernels when it is created.  Errors: MOE_EBOUNDS, MOE_ESTATE (expert never loaded). */
 int moe_stream_misses(moe_pool* pool, int layer, const moe_miss* miss_h, int n_miss,
                       void* copy_stream);
 
@@ -206,6 +220,14 @@ int moe_expert_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const i
  * all rows of h (default 5000), a shared-memory pipeline stage (default 10000).
  * Process-wide; affects later launches.  Errors: MOE_EINVAL (non-positive). */
 int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
+
+/* Tracing: when buf is a device buffer of at least 8 * 148 (8 per SM) u64,
+ * each CTA of every later moe_expert_ffn launch writes global-timer stamps (ns)
+ * of its phases: [0] start, [1] expert table built, [2] activations staged,
+ * [3] first item's weights landed, [4] gate/up items done and published,
+ * [5] first down item's h dependency met, [6] last item done, [7] end.
+ * Unwritten entries keep their old value.  NULL turns tracing off. */
+int moe_set_ffn_trace(void* buf);
 
 /* Router-weighted combine (post.smzdm.com/p/a825qpgl section 二: results merged
  * by routing weight): y[t, :] = bf16(sum over j = 0..k-1 of y_part[t, j, :]),

@@ -341,3 +341,25 @@ def test_bad_slot_index_is_reported_not_used(m):
         m.set_wait_limits(5000, 5000, 10000)
     assert int(lo.status.item()) & m._lib.STATUS_BAD_SLOT
     pool.close()
+
+
+def test_decode_layer_call_with_misses_matches_oracle(m):
+    """The public DecodeLayer call (FFN enqueued before the host drives the copy
+    engine) over steps and layers with misses."""
+    w = small("dl", "nvfp4", H=512, I=512, E=16, k=4, L=3, zipf=0.8)
+    T = 4
+    pool = m.Pool(w.H, w.I, w.E, w.k, w.L, w.fmt, 16, max_tokens=T)
+    for layer in range(w.L):
+        for e in range(w.E):
+            pool.load_expert(layer, e, weights(w, layer, e))
+    lo = m.DecodeLayer(pool, T)
+    for step in range(3):
+        for layer in range(w.L):
+            x = gen.activations(w, layer, step, T)
+            wr = gen.router_weight(w, layer)
+            b = gen.router_bias(w, layer)
+            lo(layer, bf16(x), bf16(wr), dev(b))
+            torch.cuda.synchronize()
+            check_layer(w, lo, x, wr, b, layer)
+    assert pool.stats()["misses"] > 0
+    pool.close()
