@@ -73,6 +73,7 @@ SIGNATURES = {
     "moe_dequant_slot": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_set_wait_limits": (i32, [f64, f64, f64]),
     "moe_set_ffn_trace": (i32, [vp]),
+    "moe_nvfp4_gemm": (i32, [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]),
     "moe_route_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]),
 }
 

@@ -184,6 +184,14 @@ def dequant_slot(pool, slot, key, which, out, stream=None):
         pool.handle, int(slot), int(key), int(which), _p(out), _s(stream)))
 
 
+def nvfp4_gemm(a_codes, a_scales, b_codes, b_scales, D, status, stream=None):
+    """D [M, N] fp32 = dq(A) dq(B)^T for NVFP4 A [M, K] and B [N, K] (codes uint8
+    [rows, K/2], E4M3 scales uint8 [rows, K/16]), on the tcgen05 tensor cores."""
+    M, N, K = a_codes.shape[0], b_codes.shape[0], a_codes.shape[1] * 2
+    L.check("moe_nvfp4_gemm", L.load().moe_nvfp4_gemm(
+        _p(a_codes), _p(a_scales), _p(b_codes), _p(b_scales), M, N, K, _p(D), _p(status), _s(stream)))
+
+
 def set_wait_limits(ready_ms, dep_ms, pipe_ms):
     L.check("moe_set_wait_limits", L.load().moe_set_wait_limits(float(ready_ms), float(dep_ms),
                                                                  float(pipe_ms)))

@@ -57,6 +57,7 @@ BlockLayout block_layout(const moe_config& c);
 int preload_router_kernels();
 int preload_lookup_kernels();
 int preload_ffn_kernels();
+int preload_gemm_kernels();
 
 }  // namespace moe
 

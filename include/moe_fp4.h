@@ -229,6 +229,17 @@ int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
  * Unwritten entries keep their old value.  NULL turns tracing off. */
 int moe_set_ffn_trace(void* buf);
 
+/* Block-scaled NVFP4 GEMM on the tcgen05 tensor cores (the contraction of
+ * the prefill expert FFN; post.smzdm.com/p/aomxznrn "FreeToken干的事":
+ * compute-bound prefill scheduled apart from decode).  D[M, N] (fp32,
+ * row-major) = sum_k dq(A)[m, k] * dq(B)[n, k], where A [M, K] and B [N, K] are
+ * E2M1 codes (K-contiguous, K/2 bytes per row) with E4M3 scales per 16 elements
+ * in the canonical layout [rows, K/16]; no tensor scale (apply it to D).
+ * Limits: M, N multiples of 128, K a multiple of 256, operands 16-byte aligned.
+ * Bounded device waits set bit 16 of *status (device int) on timeout. */
+int moe_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                   const uint8_t* b_scales, int M, int N, int K, float* D, int* status, void* stream);
+
 /* Router-weighted combine (post.smzdm.com/p/a825qpgl section 二: results merged
  * by routing weight): y[t, :] = bf16(sum over j = 0..k-1 of y_part[t, j, :]),
  * summed in fp32 in rank order, rounded to nearest even. */
