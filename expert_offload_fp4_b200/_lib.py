@@ -74,6 +74,9 @@ SIGNATURES = {
     "moe_set_wait_limits": (i32, [f64, f64, f64]),
     "moe_set_ffn_trace": (i32, [vp]),
     "moe_nvfp4_gemm": (i32, [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]),
+    "moe_nvfp4_quantize": (i32, [vp, i32, i32, vp, vp, vp, vp]),
+    "moe_prefill_workspace_bytes": (sz, [vp, i32]),
+    "moe_prefill_ffn": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, sz, vp, vp]),
     "moe_route_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]),
 }
 

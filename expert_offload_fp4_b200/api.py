@@ -192,6 +192,24 @@ def nvfp4_gemm(a_codes, a_scales, b_codes, b_scales, D, status, stream=None):
         _p(a_codes), _p(a_scales), _p(b_codes), _p(b_scales), M, N, K, _p(D), _p(status), _s(stream)))
 
 
+def nvfp4_quantize(x, codes, scales, sx, stream=None):
+    """Per-token NVFP4 quantisation of x [T, H] bf16 (the prefill A operand)."""
+    T, H = x.shape
+    L.check("moe_nvfp4_quantize", L.load().moe_nvfp4_quantize(
+        _p(x), T, H, _p(codes), _p(scales), _p(sx), _s(stream)))
+
+
+def prefill_workspace_bytes(pool, T):
+    return pool.lib.moe_prefill_workspace_bytes(pool.handle, int(T))
+
+
+def prefill_ffn(pool, layer, x, idx, w, slot_of, y_part, workspace, status, stream=None):
+    T = x.shape[0]
+    L.check("moe_prefill_ffn", pool.lib.moe_prefill_ffn(
+        pool.handle, int(layer), _p(x), T, _p(idx), _p(w), _p(slot_of), _p(y_part), _p(workspace),
+        workspace.numel() * workspace.element_size(), _p(status), _s(stream)))
+
+
 def set_wait_limits(ready_ms, dep_ms, pipe_ms):
     L.check("moe_set_wait_limits", L.load().moe_set_wait_limits(float(ready_ms), float(dep_ms),
                                                                  float(pipe_ms)))

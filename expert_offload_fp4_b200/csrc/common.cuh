@@ -58,6 +58,7 @@ int preload_router_kernels();
 int preload_lookup_kernels();
 int preload_ffn_kernels();
 int preload_gemm_kernels();
+int preload_prefill_kernels();
 
 }  // namespace moe
 

@@ -166,7 +166,7 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
         return rc;
     }
     if ((rc = preload_router_kernels()) || (rc = preload_lookup_kernels()) || (rc = preload_ffn_kernels()) ||
-        (rc = preload_gemm_kernels())) {
+        (rc = preload_gemm_kernels()) || (rc = preload_prefill_kernels())) {
         moe_pool_destroy(p);
         return rc;
     }

@@ -240,6 +240,31 @@ int moe_set_ffn_trace(void* buf);
 int moe_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
                    const uint8_t* b_scales, int M, int N, int K, float* D, int* status, void* stream);
 
+/* Prefill activation quantiser (the A operand of the prefill GEMMs): each
+ * token row of x [T, H] bf16 -> NVFP4 with a per-token FP32 scale
+ * S_x = amax(x_t) / (6*448), E4M3 scales per 16 elements
+ * s = E4M3(amax_block / (6 S_x)) and codes E2M1(v / (e4m3(s) S_x)), both
+ * round-to-nearest-even and saturating (all codes 0 when e4m3(s) S_x == 0).
+ * Outputs codes [T, H/2], scales [T, H/16], sx [T].  Limits: H % 256 == 0. */
+int moe_nvfp4_quantize(const void* x_bf16, int T, int H, uint8_t* codes, uint8_t* scales, float* sx,
+                       void* stream);
+
+/* Prefill expert FFN (post.smzdm.com/p/aomxznrn "FreeToken干的事": prefill is
+ * compute-bound and scheduled apart from decode).  Groups the (token, rank)
+ * pairs by expert, quantises x to NVFP4 (as moe_nvfp4_quantize), runs the
+ * gate/up GEMM on tcgen05 with a fused SiLU*up epilogue that re-quantises h to
+ * NVFP4 (tensor scale 1), then the down GEMM with a fused routing-weight
+ * epilogue: y_part[t, j, :] = w[t, j] * S_down * (W_down h)_t for expert
+ * idx[t, j] read from slot slot_of[t, j] (all chosen experts resident).
+ * NVFP4 pools only; the expert block layout must divide into rows of H/2, H/16,
+ * I/2 and I/16 bytes (MOE_EINVAL otherwise).  workspace: device memory of
+ * moe_prefill_workspace_bytes(pool, T) bytes.  Device-side waits are bounded
+ * and set bit 16 of *status (device int) on timeout.  Follow with moe_combine. */
+size_t moe_prefill_workspace_bytes(const moe_pool* pool, int T);
+int moe_prefill_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const int32_t* idx,
+                    const float* w, const int32_t* slot_of, float* y_part, void* workspace,
+                    size_t workspace_bytes, int* status, void* stream);
+
 /* Router-weighted combine (post.smzdm.com/p/a825qpgl section 二: results merged
  * by routing weight): y[t, :] = bf16(sum over j = 0..k-1 of y_part[t, j, :]),
  * summed in fp32 in rank order, rounded to nearest even. */
