@@ -46,6 +46,55 @@ def peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+FP4_PER_BF16 = 4.0   # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+
+
+def prefill_flops(w, T):
+    """Algorithmic FLOPs of the prefill expert FFN: gate+up and down over T*k rows."""
+    return 2.0 * T * w.k * w.H * (2 * w.I) + 2.0 * T * w.k * w.I * w.H
+
+
+def prefill_run(torch, m, w, T, experts, reps=5):
+    """The prefill expert FFN of one layer (all experts resident) on a T-token prompt:
+    CUDA events around moe_prefill_ffn + moe_combine, repeated."""
+    pool = m.Pool(w.H, w.I, w.E, w.k, 1, w.fmt, w.E, max_tokens=1, host_layers=1)
+    for e in range(w.E):
+        pool.load_expert(0, e, experts[e])
+    x = torch.from_numpy(gen.activations(w, 0, 0, T).view(np.int16)).cuda().view(torch.bfloat16)
+    wr = torch.from_numpy(gen.router_weight(w, 0).view(np.int16)).cuda().view(torch.bfloat16)
+    idx = torch.empty((T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((T, w.k), dtype=torch.float32, device="cuda")
+    slot_of = torch.empty_like(idx)
+    ws = torch.zeros(m.route_workspace_bytes(T, w.E), dtype=torch.uint8, device="cuda")
+    m.route(x, wr, None, w.k, 1, idx, wt, ws)
+    res = m.slot_lookup(pool, 0, idx, slot_of)
+    cs = torch.cuda.Stream()
+    m.stream_misses(pool, 0, res, cs)
+    cs.synchronize()
+    y_part = torch.empty((T, 1, w.H), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, w.H), dtype=torch.bfloat16, device="cuda")
+    work = torch.zeros(m.prefill_workspace_bytes(pool, T), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        m.prefill_ffn(pool, 0, x, idx, wt, slot_of, y_part, work, status)
+        m.combine(y_part, y)
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    e0.record(cur)
+    for _ in range(reps):
+        m.prefill_ffn(pool, 0, x, idx, wt, slot_of, y_part, work, status)
+    e1.record(cur)
+    for _ in range(reps):
+        m.combine(y_part, y)
+    e2.record(cur)
+    torch.cuda.synchronize()
+    ok = int(status.item()) == 0
+    pool.close()
+    ffn_ms = e0.elapsed_time(e1) / reps
+    return dict(ffn_ms=ffn_ms, combine_ms=e1.elapsed_time(e2) / reps, status_ok=ok)
+
+
 # ----------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -163,15 +212,35 @@ def expert_bytes_alg(w):
     return 3 * (w.H * w.I // 2 + w.H * w.I // bs)
 
 
+# ---------------------------------------------------------------- ranks
+
+def reduce_over_ranks(torch, values, device):
+    """Max over ranks of each timing (ms); the values unchanged on one rank."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def replica_value(tokens_per_rank, world, max_ms):
+    """Whole-job tokens/s of independent replicas: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (max_ms * 1e-3)
+
+
 # ---------------------------------------------------------------- decode runs
 
 def decode_run(torch, m, w, pool, T, xs_dev, wr, bias, steps, warmup, events=False, overlap=True):
     """Times `steps` decode steps (all L layers each) on the current stream."""
     lo = m.DecodeLayer(pool, T, overlap=overlap)
     cur = torch.cuda.current_stream()
+    per_layer = isinstance(wr, (list, tuple))
+    wr_of = (lambda l: wr[l]) if per_layer else (lambda l: wr)
+    b_of = (lambda l: bias[l]) if per_layer else (lambda l: bias)
     for s in range(warmup):
         for l in range(w.L):
-            lo(l, xs_dev[s % xs_dev.shape[0], l], wr, bias)
+            lo(l, xs_dev[s % xs_dev.shape[0], l], wr_of(l), b_of(l))
     torch.cuda.synchronize()
     st0 = pool.stats()
     if events:
@@ -180,7 +249,7 @@ def decode_run(torch, m, w, pool, T, xs_dev, wr, bias, steps, warmup, events=Fal
     e0.record(cur)
     for s in range(steps):
         for l in range(w.L):
-            lo(l, xs_dev[(warmup + s) % xs_dev.shape[0], l], wr, bias)
+            lo(l, xs_dev[(warmup + s) % xs_dev.shape[0], l], wr_of(l), b_of(l))
     e1.record(cur)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
@@ -284,6 +353,106 @@ def ffn_only(args, w, T):
                       "phases_us_median_max": phases}), flush=True)
 
 
+# ------------------------------------------------------- 284B decode + cache stress
+
+def load_mxfp4_store(m, w, pool, host_layers, threads=16):
+    """Generate the uniform-MXFP4 experts of host_layers layers and pack them into the
+    pool's pinned store (threads: numpy and the packing call release the GIL)."""
+    import concurrent.futures as cf
+
+    def job(he):
+        hl, e = he
+        pool.load_expert(hl, e, gen.expert_weights(w, hl, e))
+    with cf.ThreadPoolExecutor(threads) as ex:
+        list(ex.map(job, [(hl, e) for hl in range(host_layers) for e in range(w.E)]))
+
+
+def resident_layer_ms(torch, m, w, pool, xs_dev, wr, bias, reps=20):
+    """Per-layer time of route + lookup + FFN + combine with every expert a hit:
+    layer 0 of the pool made fully resident, then repeated."""
+    pool.reset()
+    idx = torch.arange(w.E, dtype=torch.int32, device="cuda").view(-1, w.k) if w.E % w.k == 0 else None
+    if idx is None:
+        ids = list(range(w.E)) + list(range(w.k - w.E % w.k))
+        idx = torch.tensor(ids, dtype=torch.int32, device="cuda").view(-1, w.k)
+    slot_of = torch.empty_like(idx)
+    cs = torch.cuda.Stream()
+    res = m.slot_lookup(pool, 0, idx, slot_of)
+    m.stream_misses(pool, 0, res, cs)
+    cs.synchronize()
+    lo = m.DecodeLayer(pool, 1)
+    for i in range(3):
+        lo(0, xs_dev[i % xs_dev.shape[0], 0], wr[0], bias[0])
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for i in range(reps):
+        lo(0, xs_dev[i % xs_dev.shape[0], 0], wr[0], bias[0])
+    e1.record(cur)
+    torch.cuda.synchronize()
+    assert lo.lookup.n_miss == 0
+    return e0.elapsed_time(e1) / reps
+
+
+def overlap_efficiency(t_wall, t_copy, t_comp):
+    """1 - (T_wall - max(T_copy, T_comp)) / min(T_copy, T_comp), clipped to [0, 1]."""
+    lo, hi = min(t_copy, t_comp), max(t_copy, t_comp)
+    if lo <= 0:
+        return None
+    return max(0.0, min(1.0, 1.0 - (t_wall - hi) / lo))
+
+
+def offload_mode(args):
+    """decode_284b (2570-slot / 32 GiB pool) and the cache-stress sweep over Zipf
+    exponent x pool fraction: tokens/s, hit rate, H2D GB/s, overlap efficiency and
+    the q* split for the pages' four machines.  One JSON line per run."""
+    import torch
+    import expert_offload_fp4_b200 as m
+    w = W.DECODE_284B
+    HL = args.host_layers
+    max_slots = max(W.n_slots(w), max(W.n_slots(W.stress_variant(0.0, p)) for p in W.STRESS_POOL))
+    pool = m.Pool(w.H, w.I, w.E, w.k, w.L, w.fmt, max_slots, max_tokens=1, host_layers=HL)
+    t0 = time.perf_counter()
+    load_mxfp4_store(m, w, pool, HL)
+    load_s = time.perf_counter() - t0
+    nbuf = 8
+    xs = np.stack([np.stack([gen.activations(w, l, s, 1) for l in range(w.L)]) for s in range(nbuf)])
+    xs_dev = torch.from_numpy(xs.view(np.int16)).cuda().view(torch.bfloat16)
+    wr = [torch.from_numpy(gen.router_weight(w, l).view(np.int16)).cuda().view(torch.bfloat16) for l in range(w.L)]
+    t_layer = resident_layer_ms(torch, m, w, pool, xs_dev, wr, [None] * w.L)
+    runs = [("decode_284b", w, W.n_slots(w), w.zipf_s, args.steps)]
+    for zs in W.STRESS_ZIPF:
+        for pf in W.STRESS_POOL:
+            v = W.stress_variant(zs, pf)
+            runs.append((v.name, v, W.n_slots(v), zs, W.STRESS_284B.steps))
+    for name, v, slots, zs, steps in runs:
+        bias = [torch.from_numpy(gen.router_bias(v, l, zs)).cuda() for l in range(w.L)]
+        pool.reset(slots)
+        r = decode_run(torch, m, w, pool, 1, xs_dev, wr, bias, steps, args.warmup, events=True,
+                       overlap=not args.no_overlap)
+        st = r["stats"]
+        copy_ms = sum(t for t, _ in r["copy"])
+        t_comp = t_layer * w.L * steps
+        m_layer = st["misses"] / (steps * w.L)
+        q = {f"{bp}/{bh}": dict(zip(("q_gpu", "q_cpu", "ratio"), m.qstar_split(int(round(m_layer)), bp, bh)))
+             for bp, bh in W.QSTAR_MACHINES}
+        line = {"mode": "offload", "run": name, "zipf_s": zs, "slots": slots,
+                "slot_frac": round(slots / (w.L * w.E), 4), "steps": steps, "warmup": args.warmup,
+                "tokens_per_s": round(steps / (r["ms"] * 1e-3), 3), "ms_per_step": round(r["ms"] / steps, 4),
+                "hit_rate": round(st["hits"] / max(1, st["unique"]), 4),
+                "misses_per_layer": round(m_layer, 3),
+                "h2d_gbs": round(st["h2d_bytes"] / (copy_ms * 1e-3) / 1e9, 2) if copy_ms > 0 else None,
+                "h2d_bytes_per_step": st["h2d_bytes"] // steps,
+                "t_wall_ms": round(r["ms"], 2), "t_copy_ms": round(copy_ms, 2), "t_comp_ms": round(t_comp, 2),
+                "overlap_efficiency": overlap_efficiency(r["ms"], copy_ms, t_comp),
+                "qstar_per_layer": q, "status": r["status"],
+                "host_store": f"{HL} distinct layer weight sets for {w.L} layer positions",
+                "store_load_s": round(load_s, 1)}
+        print(json.dumps(line), flush=True)
+    pool.close()
+
+
 # ---------------------------------------------------------------------- main
 
 def main():
@@ -295,11 +464,13 @@ def main():
     ap.add_argument("--batch", type=int, default=1, help="decode tokens per step (1, 4 or 8)")
     ap.add_argument("--all-batches", action="store_true", help="also time batches 4 and 8")
     ap.add_argument("--oracle-budget", type=float, default=10.0)
-    ap.add_argument("--mode", default="decode", choices=["decode", "ffn"],
+    ap.add_argument("--mode", default="decode", choices=["decode", "ffn", "prefill", "offload"],
                     help="ffn: only the decode FFN kernel on a small all-resident pool "
                          "(a few layers), e.g. for an ncu capture")
     ap.add_argument("--layers", type=int, default=4, help="layer positions in --mode ffn")
     ap.add_argument("--trace", action="store_true", help="--mode ffn: per-CTA phase timestamps")
+    ap.add_argument("--host-layers", type=int, default=8,
+                    help="--mode offload: distinct host copies of the 40 layers (pinned RAM)")
     ap.add_argument("--no-overlap", action="store_true",
                     help="issue miss copies before each FFN launch (for runs under ncu, which "
                          "serialises kernels)")
@@ -333,6 +504,22 @@ def main():
 
     if args.mode == "ffn":
         return ffn_only(args, w, T)
+    if args.mode == "offload":
+        return offload_mode(args)
+    if args.mode == "prefill":
+        wp = W.PREFILL_35B
+        experts = gen.expert_weights_many(wp, 0, range(wp.E))
+        import torch
+        import expert_offload_fp4_b200 as m
+        r = prefill_run(torch, m, wp, 2048, experts)
+        fl = prefill_flops(wp, 2048)
+        _, bf16_peak, kind = peaks()
+        print(json.dumps({"mode": "prefill", "workload": wp.name, "ffn_ms": round(r["ffn_ms"], 4),
+                          "combine_ms": round(r["combine_ms"], 4),
+                          "tflops": round(fl / (r["ffn_ms"] * 1e-3) / 1e12, 1),
+                          "peak_fp4_tflops": bf16_peak * FP4_PER_BF16, "status_ok": r["status_ok"]}),
+              flush=True)
+        return
 
     # inputs first (spawned generator workers), then CUDA
     experts = gen.expert_weights_many(w, 0, range(w.E))
@@ -392,18 +579,20 @@ def main():
     alg_avg = sum(alg_bytes) / len(alg_bytes)
     achieved = alg_avg / (ffn_ms * 1e-3) / 1e9
 
+    # prefill of the same layer: a 2048-token prompt, all experts resident
+    wp = W.PREFILL_35B
+    pr = prefill_run(torch, m, wp, 2048, experts)
+    pfl = prefill_flops(wp, 2048)
+    _, bf16_peak, _ = peaks()
+    fp4_peak = bf16_peak * FP4_PER_BF16
+
     # reduce over ranks: max time, summed tokens
     r = res[T]
-    ms = r["ms"]
+    ms, e2e_ms = reduce_over_ranks(torch, [r["ms"], e2e["ms"]], "cuda")
     if world > 1:
-        t = torch.tensor([ms, e2e["ms"]], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
         torch.distributed.barrier()
-    else:
-        e2e_ms = e2e["ms"]
     tokens = T * args.steps * world
-    value = tokens / (ms * 1e-3)
+    value = replica_value(T * args.steps, world, ms)
     st = r["stats"]
     copy_ms = sum(t for t, _ in r["copy"])
     h2d_gbs = st["h2d_bytes"] / (copy_ms * 1e-3) / 1e9 if copy_ms > 0 else None
@@ -429,7 +618,7 @@ def main():
                          "measured_on": "all-resident pool, same layers/inputs",
                          "launch_ms_avg": round(ffn_ms, 5),
                          "alg_bytes_per_launch_avg": int(alg_avg)},
-            "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 3), "unit": "tokens/s",
+            "e2e": {"value": round(replica_value(T * args.steps, world, e2e_ms), 3), "unit": "tokens/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
             "gpu_launches": 4 * w.L * args.steps,
             "clocks": clocks,
@@ -439,6 +628,13 @@ def main():
             "misses_per_layer": round(st["misses"] / (args.steps * w.L), 3),
             "batches": {str(b): round(b * args.steps / (res[b]["ms"] * 1e-3), 3) for b in res},
             "status": r["status"],
+            "prefill": {"workload": wp.name, "tokens": 2048, "ffn_ms": round(pr["ffn_ms"], 4),
+                        "combine_ms": round(pr["combine_ms"], 4), "flops": pfl,
+                        "tflops": round(pfl / (pr["ffn_ms"] * 1e-3) / 1e12, 1),
+                        "peak_tflops": fp4_peak,
+                        "frac": round(pfl / (pr["ffn_ms"] * 1e-3) / 1e12 / fp4_peak, 4),
+                        "peak_source": "measured bf16 x 4 (nominal FP4:BF16 ratio)",
+                        "status_ok": pr["status_ok"]},
         }
         if cb is not None:
             line["cpu_baseline"] = cb

@@ -59,6 +59,7 @@ SIGNATURES = {
     "moe_expert_block_bytes": (sz, [C.POINTER(MoeConfig)]),
     "moe_pool_load_expert": (i32, [vp, i32, i32, C.POINTER(ExpertSrc)]),
     "moe_pool_read_state": (i32, [vp, vp, vp, vp, vp]),
+    "moe_pool_reset": (i32, [vp, i32]),
     "moe_pool_stats": (i32, [vp, C.POINTER(Stats)]),
     "moe_pool_slot_ptr": (i32, [vp, i32, C.POINTER(vp), C.POINTER(sz)]),
     "moe_route_workspace_bytes": (sz, [i32, i32]),

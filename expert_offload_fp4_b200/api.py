@@ -71,6 +71,12 @@ class Pool:
         L.check("moe_pool_load_expert",
                 self.lib.moe_pool_load_expert(self.handle, int(layer), int(expert), C.byref(src)))
 
+    def reset(self, n_active_slots=None):
+        """Empty the pool and use only the first n_active_slots slots from now on."""
+        n = self.n_slots if n_active_slots is None else int(n_active_slots)
+        L.check("moe_pool_reset", self.lib.moe_pool_reset(self.handle, n))
+        self.n_active = n
+
     def read_state(self):
         sk = np.empty(self.n_slots, np.int32)
         sc = np.empty(self.n_slots, np.uint64)
@@ -203,10 +209,12 @@ def prefill_workspace_bytes(pool, T):
     return pool.lib.moe_prefill_workspace_bytes(pool.handle, int(T))
 
 
-def prefill_ffn(pool, layer, x, idx, w, slot_of, y_part, workspace, status, stream=None):
+def prefill_ffn(pool, layer, x, idx, w, slot_of, y, workspace, status, stream=None):
+    """y [T, H] fp32 (zeroed by the call) = the routed experts' FFN outputs summed
+    with their routing weights; round with combine(y.view(T, 1, H), y_bf16)."""
     T = x.shape[0]
     L.check("moe_prefill_ffn", pool.lib.moe_prefill_ffn(
-        pool.handle, int(layer), _p(x), T, _p(idx), _p(w), _p(slot_of), _p(y_part), _p(workspace),
+        pool.handle, int(layer), _p(x), T, _p(idx), _p(w), _p(slot_of), _p(y), _p(workspace),
         workspace.numel() * workspace.element_size(), _p(status), _s(stream)))
 
 

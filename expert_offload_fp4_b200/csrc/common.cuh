@@ -67,6 +67,7 @@ struct moe_pool {
     int bs;                       // elements per block scale
     moe::BlockLayout lay;
     int host_layers;
+    int n_active;                 // slots the LRU may use (<= cfg.n_slots)
     int device;
     int num_sms;
     // storage

@@ -259,7 +259,7 @@ extern "C" int moe_slot_lookup_launch(moe_pool* p, int layer, const int32_t* idx
     if (T <= 0 || k <= 0 || k > c.E || (long long)T * k > (1LL << 24)) return fail(MOE_EINVAL, "bad T/k");
     // the pool must hold every expert one call can touch, or a miss finds no victim
     const int cap = T * k < c.E ? T * k : c.E;
-    if (cap > c.n_slots) return fail(MOE_EINVAL, "slot pool smaller than the unique experts one call can touch");
+    if (cap > p->n_active) return fail(MOE_EINVAL, "slot pool smaller than the unique experts one call can touch");
     if (p->lk_pending) return fail(MOE_ESTATE, "a launched lookup has not been collected");
     cudaStream_t s = (cudaStream_t)stream;
     LookupArgs a;
@@ -267,7 +267,7 @@ extern "C" int moe_slot_lookup_launch(moe_pool* p, int layer, const int32_t* idx
     a.n = T * k;
     a.layer = layer;
     a.E = c.E;
-    a.S = c.n_slots;
+    a.S = p->n_active;
     a.slot_key = p->slot_key;
     a.slot_clock = p->slot_clock;
     a.key_slot = p->key_slot;
@@ -277,7 +277,7 @@ extern "C" int moe_slot_lookup_launch(moe_pool* p, int layer, const int32_t* idx
     a.slot_of = slot_of;
     a.out = p->lk_d;
     a.seq = ++p->lk_seq;
-    const size_t smem = size_t(2) * ((c.n_slots + 31) / 32) * sizeof(uint32_t);
+    const size_t smem = size_t(2) * ((p->n_active + 31) / 32) * sizeof(uint32_t);
     if (smem > 160 * 1024) return fail(MOE_EINVAL, "n_slots too large for the lookup kernel");
     if (!p->lk_attr_set) {
         MOE_CUDA_TRY(cudaFuncSetAttribute(lookup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));

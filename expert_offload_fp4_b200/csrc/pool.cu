@@ -107,6 +107,7 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
     p->bs = cfg->fmt == MOE_MXFP4 ? 32 : 16;
     p->lay = block_layout(*cfg);
     p->host_layers = cfg->host_layers ? cfg->host_layers : cfg->L;
+    p->n_active = cfg->n_slots;
     cudaGetDevice(&p->device);
     cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device);
     const size_t S = cfg->n_slots, LE = size_t(cfg->L) * cfg->E;
@@ -203,6 +204,25 @@ extern "C" int moe_pool_load_expert(moe_pool* p, int layer, int expert, const mo
         if (e != cudaSuccess) return cuda_fail(e, "tensor scale upload");
     }
     p->host_loaded[size_t(layer) * c.E + expert] = 1;
+    return MOE_OK;
+}
+
+extern "C" int moe_pool_reset(moe_pool* p, int n_active_slots) {
+    if (!p) return fail(MOE_EINVAL, "null pool");
+    if (n_active_slots <= 0 || n_active_slots > p->cfg.n_slots)
+        return fail(MOE_EINVAL, "reset: active slots must be in [1, n_slots]");
+    if (p->lk_pending) return fail(MOE_ESTATE, "reset: a launched lookup has not been collected");
+    const size_t S = p->cfg.n_slots, LE = size_t(p->cfg.L) * p->cfg.E;
+    MOE_CUDA_TRY(cudaDeviceSynchronize());
+    MOE_CUDA_TRY(cudaMemset(p->slot_key, 0xFF, S * sizeof(int32_t)));
+    MOE_CUDA_TRY(cudaMemset(p->slot_clock, 0, S * sizeof(unsigned long long)));
+    MOE_CUDA_TRY(cudaMemset(p->key_slot, 0xFF, LE * sizeof(int32_t)));
+    MOE_CUDA_TRY(cudaMemset(p->clock, 0, sizeof(unsigned long long)));
+    MOE_CUDA_TRY(cudaMemset(p->ticket, 0, sizeof(uint32_t)));
+    MOE_CUDA_TRY(cudaMemset(p->need, 0, S * sizeof(uint32_t)));
+    MOE_CUDA_TRY(cudaMemset(p->ready, 0, S * sizeof(uint32_t)));
+    p->n_active = n_active_slots;
+    memset(&p->stats, 0, sizeof(p->stats));
     return MOE_OK;
 }
 

@@ -12,9 +12,11 @@
 //             epilogue h = silu(S_x S_g acc_g) * (S_x S_u acc_u), quantised to
 //             NVFP4 with tensor scale 1 (A operand of GEMM2);
 //   GEMM2     per (M tile, 128 columns of H): A = quantised h, B = down rows;
-//             epilogue y_part[t, j, :] = w[t, j] * S_d * acc.
-// moe_combine then sums y_part over j.  The mainloop is the one of
-// moe_nvfp4_gemm (TMA ring, scale-atom rearrangement, tcgen05.cp + mma).
+//             epilogue y[t, :] += w[t, j] * S_d * acc (fp32 vector reductions).
+// moe_combine(y, T, 1, H) then rounds y to bf16.  The mainloop is the one of
+// moe_nvfp4_gemm (TMA ring, scale-atom rearrangement, tcgen05.cp + mma); two
+// stages per CTA so that two CTAs share an SM and one's epilogue overlaps the
+// other's mainloop.
 #include "tcgen05.cuh"
 
 namespace moe {
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(256) prefill_quant_kernel(const uint16_t* __re
 
 // ---------------------------------------------------------------- grouped GEMMs
 
-constexpr int kPStages = 4;
+constexpr int kPStages = 2;
 constexpr int kPThreads = 256;
 constexpr uint32_t kPTmemCols = 256;
 
@@ -230,7 +232,7 @@ struct GemmArgs {
     PrefillWs ws;
     const float* tscale;        // [L*E*3]
     const float* w;             // [T*k]
-    float* y_part;              // [T*k*H]
+    float* y;                   // [T*H] fp32, accumulated
     int* status;
     int layer, E, k, H, I, NT;  // NT: N tiles per M tile
     long long b_gate_row, b_up_row, b_gsf_row, b_usf_row;  // row offsets inside a slot (GEMM1)
@@ -373,22 +375,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
         } else {
             const int n0 = nt * 128;
             float coef = 0.0f;
-            size_t dst = 0;
+            float* dst = nullptr;
             if (tok >= 0) {
                 const int j = g.ws.perm_rank[row];
                 coef = g.w[tok * g.k + j] * ts[2];
-                dst = ((size_t)tok * g.k + j) * g.H + n0;
+                dst = g.y + (size_t)tok * g.H + n0;
             }
 #pragma unroll
             for (int c = 0; c < 4; c++) {
                 uint32_t r[32];
                 tmem_ld_32x32(lane_base + 32 * c, r);
                 if (tok >= 0) {
-                    float4* o = reinterpret_cast<float4*>(g.y_part + dst + 32 * c);
 #pragma unroll
                     for (int q = 0; q < 8; q++)
-                        o[q] = make_float4(coef * __uint_as_float(r[4 * q]), coef * __uint_as_float(r[4 * q + 1]),
-                                           coef * __uint_as_float(r[4 * q + 2]), coef * __uint_as_float(r[4 * q + 3]));
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                                     ::"l"(dst + 32 * c + 4 * q), "f"(coef * __uint_as_float(r[4 * q])),
+                                       "f"(coef * __uint_as_float(r[4 * q + 1])), "f"(coef * __uint_as_float(r[4 * q + 2])),
+                                       "f"(coef * __uint_as_float(r[4 * q + 3]))
+                                     : "memory");
                 }
             }
         }
@@ -459,9 +463,9 @@ extern "C" int moe_nvfp4_quantize(const void* x_bf16, int T, int H, uint8_t* cod
 }
 
 extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx,
-                               const float* w, const int32_t* slot_of, float* y_part, void* workspace,
+                               const float* w, const int32_t* slot_of, float* y, void* workspace,
                                size_t workspace_bytes, int* status, void* stream) {
-    if (!p || !x_bf16 || !idx || !w || !slot_of || !y_part || !workspace || !status)
+    if (!p || !x_bf16 || !idx || !w || !slot_of || !y || !workspace || !status)
         return fail(MOE_EINVAL, "null argument");
     const moe_config& c = p->cfg;
     if (layer < 0 || layer >= c.L) return fail(MOE_EBOUNDS, "layer outside the pool");
@@ -495,6 +499,7 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
     ws.R = PL.R;
     ws.MT = PL.MT;
     MOE_CUDA_TRY(cudaMemsetAsync(ws.perm_tok, 0xFF, size_t(PL.R) * 4, s));
+    MOE_CUDA_TRY(cudaMemsetAsync(y, 0, size_t(T) * c.H * sizeof(float), s));
     prefill_plan_kernel<<<1, 1024, 0, s>>>(idx, slot_of, T * c.k, c.E, ws, status);
     MOE_CUDA_TRY(cudaGetLastError());
     prefill_quant_kernel<<<(T * 32 + 255) / 256, 256, 0, s>>>((const uint16_t*)x_bf16, T, c.H, c.k, c.E, idx, ws,
@@ -517,7 +522,7 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
     g.ws = ws;
     g.tscale = p->tscale;
     g.w = w;
-    g.y_part = y_part;
+    g.y = y;
     g.status = status;
     g.layer = layer;
     g.E = c.E;

@@ -128,6 +128,12 @@ size_t moe_expert_block_bytes(const moe_config* cfg);
  * expert is not resident until a lookup misses it.  Errors: MOE_EBOUNDS. */
 int moe_pool_load_expert(moe_pool* pool, int layer, int expert, const moe_expert_src* src);
 
+/* Empty the slot pool (every expert back to host-only, LRU clock and tickets
+ * reset, statistics cleared) and let later lookups use only the first
+ * n_active_slots slots (1 .. n_slots).  Synchronises the device.  For sweeps of
+ * the pool size and for a cold restart; the host store is kept. */
+int moe_pool_reset(moe_pool* pool, int n_active_slots);
+
 /* Copy the LRU state to host arrays (synchronous; for checks and checkpoints):
  * slot_key_h[n_slots] (layer*E+expert or -1), slot_clock_h[n_slots],
  * key_slot_h[L*E] (slot or -1), *clock_h = global clock. */
@@ -254,15 +260,18 @@ int moe_nvfp4_quantize(const void* x_bf16, int T, int H, uint8_t* codes, uint8_t
  * pairs by expert, quantises x to NVFP4 (as moe_nvfp4_quantize), runs the
  * gate/up GEMM on tcgen05 with a fused SiLU*up epilogue that re-quantises h to
  * NVFP4 (tensor scale 1), then the down GEMM with a fused routing-weight
- * epilogue: y_part[t, j, :] = w[t, j] * S_down * (W_down h)_t for expert
- * idx[t, j] read from slot slot_of[t, j] (all chosen experts resident).
+ * combine: y[t, :] = sum_j w[t, j] * S_down * (W_down h)_t for expert idx[t, j]
+ * read from slot slot_of[t, j] (all chosen experts resident); y is [T, H] fp32,
+ * zeroed by the call and summed with fp32 vector reductions (the order of the
+ * k terms is not fixed).
  * NVFP4 pools only; the expert block layout must divide into rows of H/2, H/16,
  * I/2 and I/16 bytes (MOE_EINVAL otherwise).  workspace: device memory of
  * moe_prefill_workspace_bytes(pool, T) bytes.  Device-side waits are bounded
- * and set bit 16 of *status (device int) on timeout.  Follow with moe_combine. */
+ * and set bit 16 of *status (device int) on timeout.  moe_combine(y, T, 1, H, y_bf16)
+ * rounds the result to bf16. */
 size_t moe_prefill_workspace_bytes(const moe_pool* pool, int T);
 int moe_prefill_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const int32_t* idx,
-                    const float* w, const int32_t* slot_of, float* y_part, void* workspace,
+                    const float* w, const int32_t* slot_of, float* y, void* workspace,
                     size_t workspace_bytes, int* status, void* stream);
 
 /* Router-weighted combine (post.smzdm.com/p/a825qpgl section 二: results merged

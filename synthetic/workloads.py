@@ -64,9 +64,10 @@ DECODE_284B = Workload(
     notes="Zipf permutation re-drawn per layer; slot pool capped at 32 GiB")
 
 PREFILL_35B = Workload(
-    name="prefill_35b_a3b_t2048", H=2048, I=768, E=128, k=8, L=1, fmt=NVFP4, seed=4,
+    name="prefill_35b_a3b_t2048", H=2048, I=768, E=128, k=8, L=1, fmt=NVFP4, seed=2,
     batches=(2048,), steps=1, zipf_s=0.0, weight_recipe="normal", sigma=0.02,
-    notes="2048-token prompt on the decode_35b layer shape, all experts resident")
+    notes="2048-token prompt on the decode_35b layer (same weights), no routing bias, "
+          "all experts resident")
 
 STRESS_284B = Workload(
     name="stress_284b", H=4096, I=2048, E=256, k=6, L=40, fmt=MXFP4, seed=5,

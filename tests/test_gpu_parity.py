@@ -363,3 +363,27 @@ def test_decode_layer_call_with_misses_matches_oracle(m):
             check_layer(w, lo, x, wr, b, layer)
     assert pool.stats()["misses"] > 0
     pool.close()
+
+
+def test_pool_reset_restricts_active_slots(m):
+    """After a reset to n active slots the LRU behaves as a fresh n-slot pool."""
+    E, k, L = 32, 4, 2
+    pool = m.Pool(256, 256, E, k, L, "mxfp4", 24, max_tokens=2)
+    rng = np.random.default_rng(3)
+    slot_of = torch.empty((2, k), dtype=torch.int32, device="cuda")
+    for _ in range(10):
+        idx = np.stack([rng.choice(E, k, replace=False) for _ in range(2)]).astype(np.int32)
+        m.slot_lookup(pool, 0, dev(idx), slot_of)
+    pool.reset(8)
+    ref = oracle.LRU(8, L, E)
+    for step in range(30):
+        layer = step % L
+        idx = np.stack([rng.choice(E, k, replace=False) for _ in range(2)]).astype(np.int32)
+        res = m.slot_lookup(pool, layer, dev(idx), slot_of)
+        r = ref.step(layer, idx)
+        assert [s for _, s, _, _ in res.miss_list()] == r["miss_slot"].tolist()
+        assert np.array_equal(slot_of.cpu().numpy(), r["slot_of"])
+        assert slot_of.cpu().numpy().max() < 8
+    st = pool.stats()
+    assert st["lookups"] == 30
+    pool.close()

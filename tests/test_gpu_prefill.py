@@ -72,12 +72,12 @@ def run_prefill(m, w, T, experts, layer=0, step=0):
     cs = torch.cuda.Stream()
     m.stream_misses(pool, 0, res, cs)
     cs.synchronize()
-    y_part = torch.zeros((T, w.k, w.H), dtype=torch.float32, device="cuda")
+    yacc = torch.full((T, w.H), float("nan"), dtype=torch.float32, device="cuda")
     work = torch.zeros(m.prefill_workspace_bytes(pool, T), dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    m.prefill_ffn(pool, 0, xd, idx, wt, slot_of, y_part, work, status)
+    m.prefill_ffn(pool, 0, xd, idx, wt, slot_of, yacc, work, status)
     y = torch.empty((T, w.H), dtype=torch.bfloat16, device="cuda")
-    m.combine(y_part, y)
+    m.combine(yacc.view(T, 1, w.H), y)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     out = dict(x=x, wr=wr, b=b, idx=idx.cpu().numpy(), w=wt.cpu().numpy(), y=y.float().cpu().numpy())
