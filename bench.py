@@ -416,7 +416,7 @@ def offload_mode(args):
     t0 = time.perf_counter()
     load_mxfp4_store(m, w, pool, HL)
     load_s = time.perf_counter() - t0
-    nbuf = 8
+    nbuf = args.warmup + max(args.steps, W.STRESS_284B.steps)   # a fresh input for every step
     xs = np.stack([np.stack([gen.activations(w, l, s, 1) for l in range(w.L)]) for s in range(nbuf)])
     xs_dev = torch.from_numpy(xs.view(np.int16)).cuda().view(torch.bfloat16)
     wr = [torch.from_numpy(gen.router_weight(w, l).view(np.int16)).cuda().view(torch.bfloat16) for l in range(w.L)]
@@ -533,7 +533,7 @@ def main():
     m._lib.load()
 
     hbm_peak, _, peak_kind = peaks()
-    nbuf = 16
+    nbuf = args.warmup + args.steps           # a fresh input for every step
     xs = np.stack([np.stack([gen.activations(w, l, s, 8) for l in range(w.L)]) for s in range(nbuf)])
     wr = torch.from_numpy(gen.router_weight(w, 0).view(np.int16)).cuda().view(torch.bfloat16)
     bias = torch.from_numpy(gen.router_bias(w, 0)).cuda()

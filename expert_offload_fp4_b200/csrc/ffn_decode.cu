@@ -189,6 +189,55 @@ __device__ __forceinline__ void chunk_dot(const uint8_t* code, const uint8_t* sc
     }
 }
 
+// Gate and up rows of one chunk together: the activation chunk of each token is
+// loaded once and the eight f16x2 chains (4 per row) run interleaved.
+template <int FMT, int MT>
+__device__ __forceinline__ void chunk_dot_pair(const uint8_t* gcode, const uint8_t* gscl, const uint8_t* ucode,
+                                               const uint8_t* uscl, int c, int cpr, const __half* const* act,
+                                               int M, float (&ag)[MT], float (&au)[MT]) {
+    uint32_t wg[16], wu[16];
+    decode_e2m1_x2(*reinterpret_cast<const uint4*>(gcode + 16 * c), wg);
+    decode_e2m1_x2(*reinterpret_cast<const uint4*>(ucode + 16 * c), wu);
+    float g0, g1, u0, u1;
+    if (FMT == MOE_NVFP4) {
+        const float2 sg = e4m3x2_to_f32((uint32_t)gscl[2 * c] | ((uint32_t)gscl[2 * c + 1] << 8));
+        const float2 su = e4m3x2_to_f32((uint32_t)uscl[2 * c] | ((uint32_t)uscl[2 * c + 1] << 8));
+        g0 = sg.x; g1 = sg.y; u0 = su.x; u1 = su.y;
+    } else {
+        g0 = g1 = e8m0_to_f32(gscl[c]);
+        u0 = u1 = e8m0_to_f32(uscl[c]);
+    }
+#pragma unroll
+    for (int m = 0; m < MT; m++) {
+        if (m >= M) break;
+        const uint4* xp = reinterpret_cast<const uint4*>(act[m]) + c;
+        const uint4 x0 = xp[0], x1 = xp[cpr], x2 = xp[2 * cpr], x3 = xp[3 * cpr];
+        const uint32_t xv[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                 x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+        uint32_t ga = 0u, gb = 0u, gc = 0u, gd = 0u, ua = 0u, ub = 0u, uc = 0u, ud = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            ga = hfma2_u32(wg[i], xv[i], ga);
+            ua = hfma2_u32(wu[i], xv[i], ua);
+            gb = hfma2_u32(wg[i + 1], xv[i + 1], gb);
+            ub = hfma2_u32(wu[i + 1], xv[i + 1], ub);
+            gc = hfma2_u32(wg[8 + i], xv[8 + i], gc);
+            uc = hfma2_u32(wu[8 + i], xv[8 + i], uc);
+            gd = hfma2_u32(wg[9 + i], xv[9 + i], gd);
+            ud = hfma2_u32(wu[9 + i], xv[9 + i], ud);
+        }
+        if (FMT == MOE_NVFP4) {
+            ag[m] = fmaf(f16x2_sum(ga) + f16x2_sum(gb), g0, ag[m]);
+            ag[m] = fmaf(f16x2_sum(gc) + f16x2_sum(gd), g1, ag[m]);
+            au[m] = fmaf(f16x2_sum(ua) + f16x2_sum(ub), u0, au[m]);
+            au[m] = fmaf(f16x2_sum(uc) + f16x2_sum(ud), u1, au[m]);
+        } else {
+            ag[m] = fmaf((f16x2_sum(ga) + f16x2_sum(gb)) + (f16x2_sum(gc) + f16x2_sum(gd)), g0, ag[m]);
+            au[m] = fmaf((f16x2_sum(ua) + f16x2_sum(ub)) + (f16x2_sum(uc) + f16x2_sum(ud)), u0, au[m]);
+        }
+    }
+}
+
 template <int MT>
 __device__ __forceinline__ void group_reduce(float (&acc)[MT], int G) {
 #pragma unroll
@@ -251,6 +300,50 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
     const unsigned long long codeA = (unsigned long long)a.H / 2, sclA = (unsigned long long)a.H / bs;
     const unsigned long long codeB = (unsigned long long)a.I / 2, sclB = (unsigned long long)a.I / bs;
 
+    // ---- prologue 1 (before the previous kernel of the stream finishes): barriers
+    // and the activations, which predate the router: per-token power-of-two
+    // scale, f16, piece-major rows, 16-byte loads (8 bf16), a shared per-token max
+    // first (in hinv, free until the down projection)
+    const int cprA = a.H / 32, cprB = a.I / 32;
+    {
+        unsigned* tok_amax = reinterpret_cast<unsigned*>(hinv);
+        if (tid < a.T) tok_amax[tid] = 0u;
+        __syncthreads();
+        const int nvec = a.T * a.H / 8;
+        for (int v = tid; v < nvec; v += blockDim.x) {
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(a.x) + v);
+            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+            float mx = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(u[i] << 16)), fabsf(__uint_as_float(u[i] & 0xFFFF0000u))));
+            atomicMax(tok_amax + (v * 8) / a.H, __float_as_uint(mx));
+        }
+        __syncthreads();
+        for (int v = tid; v < nvec; v += blockDim.x) {
+            const int t = (v * 8) / a.H, h = v * 8 - t * a.H;
+            const float sc = act_scale(__uint_as_float(tok_amax[t]));
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(a.x) + v);
+            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                f[2 * i] = __uint_as_float(u[i] << 16) * sc;
+                f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u) * sc;
+            }
+            // one piece: f16x2 words (0,4), (1,5), (2,6), (3,7)
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const __half2 h2 = __floats2half2_rn(f[i], f[i + 4]);
+                o[i] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            *reinterpret_cast<uint4*>(xs + t * a.H + act_index(h, cprA)) = make_uint4(o[0], o[1], o[2], o[3]);
+            if (h == 0) xinv[t] = 1.0f / sc;
+        }
+    }
+    // ---- the slot lookup's outputs (slot_of, tickets) are needed from here on
+    pdl_wait();
     // ---- prologue: barriers, groups, activations (parallel; the stage ring is
     // still unused, so its first bytes hold the per-(token, rank) scratch)
     int* e_s = reinterpret_cast<int*>(stages);            // [n] expert or -1
@@ -267,6 +360,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
         }
         fence_mbar_init();
     }
+    __syncthreads();   // activation staging above used hinv; the table below uses the stage ring
     if (tid < n) {
         const int e = a.idx[tid], sl = a.slot_of[tid];
         int bad = 0;
@@ -330,49 +424,6 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
         if (lane == 0) s_misc[0] = c;
     }
     __syncthreads();
-    // from here the producer warp streams weights while the consumers stage the
-    // activations: per-token power-of-two scale, f16, piece-major rows, 16-byte
-    // loads (8 bf16), a shared per-token max first (in hinv, free until the
-    // down projection)
-    const int cprA = a.H / 32, cprB = a.I / 32;
-    if (warp < kNC) {
-        unsigned* tok_amax = reinterpret_cast<unsigned*>(hinv);
-        if (tid < a.T) tok_amax[tid] = 0u;
-        named_sync(2, kNC * 32);
-        const int nvec = a.T * a.H / 8;
-        for (int v = tid; v < nvec; v += kNC * 32) {
-            const uint4 q = __ldg(reinterpret_cast<const uint4*>(a.x) + v);
-            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
-            float mx = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; i++)
-                mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(u[i] << 16)), fabsf(__uint_as_float(u[i] & 0xFFFF0000u))));
-            atomicMax(tok_amax + (v * 8) / a.H, __float_as_uint(mx));
-        }
-        named_sync(2, kNC * 32);
-        for (int v = tid; v < nvec; v += kNC * 32) {
-            const int t = (v * 8) / a.H, h = v * 8 - t * a.H;
-            const float sc = act_scale(__uint_as_float(tok_amax[t]));
-            const uint4 q = __ldg(reinterpret_cast<const uint4*>(a.x) + v);
-            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
-            float f[8];
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                f[2 * i] = __uint_as_float(u[i] << 16) * sc;
-                f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u) * sc;
-            }
-            // one piece: f16x2 words (0,4), (1,5), (2,6), (3,7)
-            uint32_t o[4];
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const __half2 h2 = __floats2half2_rn(f[i], f[i + 4]);
-                o[i] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            *reinterpret_cast<uint4*>(xs + t * a.H + act_index(h, cprA)) = make_uint4(o[0], o[1], o[2], o[3]);
-            if (h == 0) xinv[t] = 1.0f / sc;
-        }
-        named_sync(2, kNC * 32);
-    }
     if (trace && tid == 0) trace[2] = globaltimer();
     const int ng = s_misc[0];
     const int nA_per = a.I / a.RA, nB_per = a.H / a.RB;
@@ -537,10 +588,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                         const uint8_t* uc = sb + m.codes1 + (size_t)p * codeA;
                         const uint8_t* us = sb + m.scl1 + m.scl1_in + (size_t)p * sclA;
 #pragma unroll 2
-                        for (int c = gl; c < cprA; c += GA) {
-                            chunk_dot<FMT, MT>(gc, gs, c, cprA, act, M, ag);
-                            chunk_dot<FMT, MT>(uc, us, c, cprA, act, M, au);
-                        }
+                        for (int c = gl; c < cprA; c += GA)
+                            chunk_dot_pair<FMT, MT>(gc, gs, uc, us, c, cprA, act, M, ag, au);
                     }
                     group_reduce<MT>(ag, GA);
                     group_reduce<MT>(au, GA);
@@ -754,6 +803,24 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     if (per_sm < 1) return fail(MOE_EINVAL, "decode FFN kernel does not fit on an SM");
     const int items_max = a.T * a.k * (c.I / a.RA + c.H / a.RB);
     const int grid = std::max(1, std::min(p->num_sms * per_sm, items_max));
+    static int pdl_ok = 1;   // cleared if the driver rejects cooperative + programmatic launch
+    if (pdl_ok) {
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(grid);
+        lc.blockDim = dim3(kFfnThreads);
+        lc.dynamicSmemBytes = smem;
+        lc.stream = s;
+        cudaLaunchAttribute at[2];
+        at[0].id = cudaLaunchAttributeCooperative;
+        at[0].val.cooperative = 1;
+        at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[1].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = at;
+        lc.numAttrs = 2;
+        if (cudaLaunchKernelEx(&lc, kern, a) == cudaSuccess) return MOE_OK;
+        cudaGetLastError();
+        pdl_ok = 0;
+    }
     void* args[] = {(void*)&a};
     MOE_CUDA_TRY(cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kFfnThreads), args, smem, s));
     return MOE_OK;

@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(LookupArgs a) {
     __shared__ int s_wslot[32];
     extern __shared__ uint32_t bits[];  // pinned [ceil(S/32)], then victim [ceil(S/32)]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();      // idx comes from the router
+    pdl_trigger();   // the expert FFN may launch and stage its activations meanwhile
     const int nwords = (a.S + 31) / 32;
     uint32_t* pinned = bits;
     uint32_t* victim = bits + nwords;
@@ -283,8 +285,19 @@ extern "C" int moe_slot_lookup_launch(moe_pool* p, int layer, const int32_t* idx
         MOE_CUDA_TRY(cudaFuncSetAttribute(lookup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
         p->lk_attr_set = 1;
     }
-    lookup_kernel<<<1, kLookupThreads, smem, s>>>(a);
-    MOE_CUDA_TRY(cudaGetLastError());
+    {
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(1);
+        lc.blockDim = dim3(kLookupThreads);
+        lc.dynamicSmemBytes = smem;
+        lc.stream = s;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = at;
+        lc.numAttrs = 1;
+        MOE_CUDA_TRY(cudaLaunchKernelEx(&lc, lookup_kernel, a));
+    }
     MOE_CUDA_TRY(cudaEventRecord(p->lk_event, s));
     p->lk_pending = 1;
     return MOE_OK;

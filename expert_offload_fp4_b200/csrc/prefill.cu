@@ -14,9 +14,8 @@
 //   GEMM2     per (M tile, 128 columns of H): A = quantised h, B = down rows;
 //             epilogue y[t, :] += w[t, j] * S_d * acc (fp32 vector reductions).
 // moe_combine(y, T, 1, H) then rounds y to bf16.  The mainloop is the one of
-// moe_nvfp4_gemm (TMA ring, scale-atom rearrangement, tcgen05.cp + mma); two
-// stages per CTA so that two CTAs share an SM and one's epilogue overlaps the
-// other's mainloop.
+// moe_nvfp4_gemm (TMA ring, scale-atom rearrangement, tcgen05.cp + mma), made
+// persistent with two TMEM accumulators (see grouped_gemm_kernel).
 #include "tcgen05.cuh"
 
 namespace moe {
@@ -46,6 +45,26 @@ __device__ __forceinline__ uint32_t e2m1_pair(float lo, float hi) {
     uint32_t b;
     asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }" : "=r"(b) : "f"(hi), "f"(lo));
     return b;
+}
+
+// h's block quantiser in the gate/up epilogue: the same steps with a reciprocal
+// multiply (h is re-rounded to FP4, so the last bit of the quotient is immaterial).
+__device__ __forceinline__ void quant_block16_fast(const float (&v)[16], uint32_t (&codes)[2], uint32_t& scale) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[i]));
+    const uint32_t sc = e4m3_code(amax * (1.0f / 6.0f));
+    const float q = e4m3_value(sc);
+    codes[0] = codes[1] = 0u;
+    if (q != 0.0f) {
+        const float rq = __frcp_rn(q);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            codes[0] |= e2m1_pair(v[i] * rq, v[i + 1] * rq) << (4 * i);
+            codes[1] |= e2m1_pair(v[8 + i] * rq, v[8 + i + 1] * rq) << (4 * i);
+        }
+    }
+    scale = sc;
 }
 
 // One 16-element block: scale s = E4M3(amax / (6 S)), q = e4m3(s) * S,
@@ -201,9 +220,9 @@ __global__ void __launch_bounds__(256) prefill_quant_kernel(const uint16_t* __re
 
 // ---------------------------------------------------------------- grouped GEMMs
 
-constexpr int kPStages = 2;
+constexpr int kPStages = 5;
 constexpr int kPThreads = 256;
-constexpr uint32_t kPTmemCols = 256;
+constexpr uint32_t kPTmemCols = 512;        // 2 accumulators x 128 + 5 stages x 32 scale columns
 
 struct PSmem {
     static constexpr int a_codes = 0;
@@ -212,8 +231,8 @@ struct PSmem {
     static constexpr int b_sf = a_sf + kPStages * 2048;
     static constexpr int a_atom = b_sf + kPStages * 2048;
     static constexpr int b_atom = a_atom + kPStages * 2048;
-    static constexpr int bars = b_atom + kPStages * 2048;
-    static constexpr int tmem_slot = bars + (3 * kPStages + 1) * 8;
+    static constexpr int bars = b_atom + kPStages * 2048;       // full, sfready, empty [stage]; accf, acce [2]
+    static constexpr int tmem_slot = bars + (3 * kPStages + 4) * 8;
     static constexpr int total = tmem_slot + 16;
 };
 
@@ -241,27 +260,29 @@ struct GemmArgs {
     unsigned long long limit_ns;
 };
 
+// Persistent, warp-specialised grouped GEMM over the (M tile, N tile) list of
+// this call; CTA c takes tiles c, c + grid, ...  Warp 0 streams every tile's K
+// steps through the stage ring without pausing between tiles; warp 2 turns the
+// scale rows into scale-factor atoms; warp 1 issues the MMAs into one of two
+// TMEM accumulators, so warps 4-7 drain tile i while tile i+1 is multiplied.
 // MODE 1: gate/up with the SiLU * up + NVFP4 epilogue; MODE 2: down with the
-// routing-weight epilogue.
+// routing-weight reduction into y.
 template <int MODE>
 __global__ void __launch_bounds__(kPThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_asf,
                     const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_bsf,
                     const GemmArgs g) {
-    const int mt = blockIdx.x / g.NT, nt = blockIdx.x % g.NT;
-    if (mt >= *g.ws.n_mtiles) return;                        // beyond this call's tiles
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + PSmem::bars);
     uint64_t* sfready = full + kPStages;
     uint64_t* empty = sfready + kPStages;
-    uint64_t* accf = empty + kPStages;
+    uint64_t* accf = empty + kPStages;     // [2]
+    uint64_t* acce = accf + 2;             // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + PSmem::tmem_slot);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = g.ws.tile_expert[mt], row0 = g.ws.tile_row0[mt];
-    const int slot = g.ws.slot_e[e];
-    const int K = MODE == 1 ? g.H : g.I;
-    const int KT = K / 256;
+    const int n_tiles = *g.ws.n_mtiles * g.NT;
+    const int KT = (MODE == 1 ? g.H : g.I) / 256;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPStages; s++) {
@@ -269,7 +290,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
             mbar_init(&sfready[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accf, 1);
+        mbar_init(&accf[0], 1);
+        mbar_init(&accf[1], 1);
+        mbar_init(&acce[0], 4);
+        mbar_init(&acce[1], 4);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, kPTmemCols);
@@ -280,123 +304,147 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
 
     if (warp == 0) {
         if (lane == 0) {
-            const long long sbase = (long long)slot * g.b_rows_per_slot;
-            const long long sfbase = (long long)slot * g.b_sf_rows_per_slot;
-            for (int kt = 0; kt < KT; kt++) {
-                const int s = kt % kPStages, r = kt / kPStages;
-                if (!mbar_wait(&empty[s], (r & 1) ^ 1, g.limit_ns)) atomicOr(g.status, 1 << 16);
-                mbar_arrive_expect_tx(&full[s], 16384 * 2 + 2048 * 2);
-                uint8_t* bc = sm + PSmem::b_codes + s * 16384;
-                uint8_t* bs = sm + PSmem::b_sf + s * 2048;
-                tma_load_2d(sm + PSmem::a_codes + s * 16384, &map_a, kt * 128, row0, &full[s]);
-                tma_load_2d(sm + PSmem::a_sf + s * 2048, &map_asf, kt * 16, row0, &full[s]);
-                if (MODE == 1) {
-                    const int i0 = nt * 64;
-                    tma_load_2d(bc, &map_b, kt * 128, (int)(sbase + g.b_gate_row + i0), &full[s]);
-                    tma_load_2d(bc + 8192, &map_b, kt * 128, (int)(sbase + g.b_up_row + i0), &full[s]);
-                    tma_load_2d(bs, &map_bsf, kt * 16, (int)(sfbase + g.b_gsf_row + i0), &full[s]);
-                    tma_load_2d(bs + 1024, &map_bsf, kt * 16, (int)(sfbase + g.b_usf_row + i0), &full[s]);
-                } else {
-                    const int n0 = nt * 128;
-                    tma_load_2d(bc, &map_b, kt * 128, (int)(sbase + g.d_row + n0), &full[s]);
-                    tma_load_2d(bs, &map_bsf, kt * 16, (int)(sfbase + g.d_sf_row + n0), &full[s]);
+            int it = 0;
+            for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+                const int mt = tile / g.NT, nt = tile % g.NT;
+                const int e = g.ws.tile_expert[mt], row0 = g.ws.tile_row0[mt];
+                const long long slot = g.ws.slot_e[e];
+                const long long sbase = slot * g.b_rows_per_slot, sfbase = slot * g.b_sf_rows_per_slot;
+                for (int kt = 0; kt < KT; kt++, it++) {
+                    const int s = it % kPStages, r = it / kPStages;
+                    if (!mbar_wait(&empty[s], (r & 1) ^ 1, g.limit_ns)) atomicOr(g.status, 1 << 16);
+                    mbar_arrive_expect_tx(&full[s], 16384 * 2 + 2048 * 2);
+                    uint8_t* bc = sm + PSmem::b_codes + s * 16384;
+                    uint8_t* bs = sm + PSmem::b_sf + s * 2048;
+                    tma_load_2d(sm + PSmem::a_codes + s * 16384, &map_a, kt * 128, row0, &full[s]);
+                    tma_load_2d(sm + PSmem::a_sf + s * 2048, &map_asf, kt * 16, row0, &full[s]);
+                    if (MODE == 1) {
+                        const int i0 = nt * 64;
+                        tma_load_2d(bc, &map_b, kt * 128, (int)(sbase + g.b_gate_row + i0), &full[s]);
+                        tma_load_2d(bc + 8192, &map_b, kt * 128, (int)(sbase + g.b_up_row + i0), &full[s]);
+                        tma_load_2d(bs, &map_bsf, kt * 16, (int)(sfbase + g.b_gsf_row + i0), &full[s]);
+                        tma_load_2d(bs + 1024, &map_bsf, kt * 16, (int)(sfbase + g.b_usf_row + i0), &full[s]);
+                    } else {
+                        const int n0 = nt * 128;
+                        tma_load_2d(bc, &map_b, kt * 128, (int)(sbase + g.d_row + n0), &full[s]);
+                        tma_load_2d(bs, &map_bsf, kt * 16, (int)(sfbase + g.d_sf_row + n0), &full[s]);
+                    }
                 }
             }
         }
     } else if (warp == 2) {
-        for (int kt = 0; kt < KT; kt++) {
-            const int s = kt % kPStages, r = kt / kPStages;
-            if (!mbar_wait(&full[s], r & 1, g.limit_ns) && lane == 0) atomicOr(g.status, 1 << 16);
-            p_arrange_sf(sm + PSmem::a_sf + s * 2048, sm + PSmem::a_atom + s * 2048, lane);
-            p_arrange_sf(sm + PSmem::b_sf + s * 2048, sm + PSmem::b_atom + s * 2048, lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sfready[s]);
+        int it = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            for (int kt = 0; kt < KT; kt++, it++) {
+                const int s = it % kPStages, r = it / kPStages;
+                if (!mbar_wait(&full[s], r & 1, g.limit_ns) && lane == 0) atomicOr(g.status, 1 << 16);
+                p_arrange_sf(sm + PSmem::a_sf + s * 2048, sm + PSmem::a_atom + s * 2048, lane);
+                p_arrange_sf(sm + PSmem::b_sf + s * 2048, sm + PSmem::b_atom + s * 2048, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfready[s]);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_fp4(128, 128, false);
-            for (int kt = 0; kt < KT; kt++) {
-                const int s = kt % kPStages, r = kt / kPStages;
-                if (!mbar_wait(&sfready[s], r & 1, g.limit_ns)) atomicOr(g.status, 1 << 16);
+            int it = 0, tc = 0;
+            for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, tc++) {
+                const int a = tc & 1, ra = tc >> 1;
+                if (!mbar_wait(&acce[a], (ra & 1) ^ 1, g.limit_ns)) atomicOr(g.status, 1 << 16);
                 tc_fence_after();
-                const uint32_t sfa = tbase + 128 + s * 32, sfb = sfa + 16;
+                const uint32_t acc = tbase + 128 * a;
+                for (int kt = 0; kt < KT; kt++, it++) {
+                    const int s = it % kPStages, r = it / kPStages;
+                    if (!mbar_wait(&sfready[s], r & 1, g.limit_ns)) atomicOr(g.status, 1 << 16);
+                    tc_fence_after();
+                    const uint32_t sfa = tbase + 256 + s * 32, sfb = sfa + 16;
 #pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    tmem_cp_sf_atom(sfa + 4 * i, smem_desc(sm + PSmem::a_atom + s * 2048 + 512 * i, 16, 128, 0));
-                    tmem_cp_sf_atom(sfb + 4 * i, smem_desc(sm + PSmem::b_atom + s * 2048 + 512 * i, 16, 128, 0));
+                    for (int i = 0; i < 4; i++) {
+                        tmem_cp_sf_atom(sfa + 4 * i, smem_desc(sm + PSmem::a_atom + s * 2048 + 512 * i, 16, 128, 0));
+                        tmem_cp_sf_atom(sfb + 4 * i, smem_desc(sm + PSmem::b_atom + s * 2048 + 512 * i, 16, 128, 0));
+                    }
+                    const uint64_t ad = smem_desc(sm + PSmem::a_codes + s * 16384, 16, 1024, 2);
+                    const uint64_t bd = smem_desc(sm + PSmem::b_codes + s * 16384, 16, 1024, 2);
+#pragma unroll
+                    for (int i = 0; i < 4; i++)
+                        mma_nvfp4(acc, ad + 2 * i, bd + 2 * i, idesc, sfa + 4 * i, sfb + 4 * i,
+                                  (kt > 0 || i > 0) ? 1u : 0u);
+                    tc_commit(&empty[s]);
                 }
-                const uint64_t ad = smem_desc(sm + PSmem::a_codes + s * 16384, 16, 1024, 2);
-                const uint64_t bd = smem_desc(sm + PSmem::b_codes + s * 16384, 16, 1024, 2);
-#pragma unroll
-                for (int i = 0; i < 4; i++)
-                    mma_nvfp4(tbase, ad + 2 * i, bd + 2 * i, idesc, sfa + 4 * i, sfb + 4 * i,
-                              (kt > 0 || i > 0) ? 1u : 0u);
-                tc_commit(&empty[s]);
+                tc_commit(&accf[a]);
             }
-            tc_commit(accf);
         }
         __syncwarp();
     } else if (warp >= 4) {
         const int q4 = warp - 4;
-        if (!mbar_wait(accf, 0, g.limit_ns) && lane == 0) atomicOr(g.status, 1 << 16);
-        tc_fence_after();
-        const int row = row0 + 32 * q4 + lane;
-        const int tok = g.ws.perm_tok[row];
-        const uint32_t lane_base = tbase + ((uint32_t)(32 * q4) << 16);
-        const float* ts = g.tscale + ((size_t)g.layer * g.E + e) * 3;
-        if (MODE == 1) {
-            const float sx = g.ws.perm_sx[row];
-            const float cg = sx * ts[0], cu = sx * ts[1];
-            for (int half = 0; half < 2; half++) {
-                uint32_t rg[32], ru[32];
-                tmem_ld_32x32(lane_base + 32 * half, rg);
-                tmem_ld_32x32(lane_base + 64 + 32 * half, ru);
-                if (tok >= 0) {
-                    // h for 32 columns of I, then two NVFP4 blocks with tensor scale 1
-                    const int i0 = nt * 64 + 32 * half;
+        int tc = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, tc++) {
+            const int a = tc & 1, ra = tc >> 1;
+            const int mt = tile / g.NT, nt = tile % g.NT;
+            const int e = g.ws.tile_expert[mt], row0 = g.ws.tile_row0[mt];
+            if (!mbar_wait(&accf[a], ra & 1, g.limit_ns) && lane == 0) atomicOr(g.status, 1 << 16);
+            tc_fence_after();
+            const int row = row0 + 32 * q4 + lane;
+            const int tok = g.ws.perm_tok[row];
+            const uint32_t lane_base = tbase + 128 * a + ((uint32_t)(32 * q4) << 16);
+            const float* ts = g.tscale + ((size_t)g.layer * g.E + e) * 3;
+            if (MODE == 1) {
+                const float sx = tok >= 0 ? g.ws.perm_sx[row] : 0.0f;
+                const float cg = sx * ts[0], cu = sx * ts[1];
+                for (int half = 0; half < 2; half++) {
+                    uint32_t rg[32], ru[32];
+                    tmem_ld_32x32(lane_base + 32 * half, rg);
+                    tmem_ld_32x32(lane_base + 64 + 32 * half, ru);
+                    if (tok >= 0) {
+                        // h for 32 columns of I, then two NVFP4 blocks with tensor scale 1
+                        const int i0 = nt * 64 + 32 * half;
 #pragma unroll
-                    for (int b = 0; b < 2; b++) {
-                        float hv[16];
+                        for (int b = 0; b < 2; b++) {
+                            float hv[16];
 #pragma unroll
-                        for (int c = 0; c < 16; c++) {
-                            const float gv = __uint_as_float(rg[16 * b + c]) * cg;
-                            const float uv = __uint_as_float(ru[16 * b + c]) * cu;
-                            hv[c] = gv / (1.0f + expf(-gv)) * uv;
+                            for (int c = 0; c < 16; c++) {
+                                const float gv = __uint_as_float(rg[16 * b + c]) * cg;
+                                const float uv = __uint_as_float(ru[16 * b + c]) * cu;
+                                hv[c] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+                            }
+                            uint32_t codes[2], sc;
+                            quant_block16_fast(hv, codes, sc);
+                            *reinterpret_cast<uint2*>(g.ws.hq + (size_t)row * (g.I / 2) + (i0 + 16 * b) / 2) =
+                                make_uint2(codes[0], codes[1]);
+                            g.ws.hsf[(size_t)row * (g.I / 16) + (i0 + 16 * b) / 16] = (uint8_t)sc;
                         }
-                        uint32_t codes[2], sc;
-                        quant_block16(hv, 1.0f, codes, sc);
-                        *reinterpret_cast<uint2*>(g.ws.hq + (size_t)row * (g.I / 2) + (i0 + 16 * b) / 2) =
-                            make_uint2(codes[0], codes[1]);
-                        g.ws.hsf[(size_t)row * (g.I / 16) + (i0 + 16 * b) / 16] = (uint8_t)sc;
+                    }
+                }
+            } else {
+                const int n0 = nt * 128;
+                float coef = 0.0f;
+                float* dst = nullptr;
+                if (tok >= 0) {
+                    const int j = g.ws.perm_rank[row];
+                    coef = g.w[tok * g.k + j] * ts[2];
+                    dst = g.y + (size_t)tok * g.H + n0;
+                }
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    uint32_t r[32];
+                    tmem_ld_32x32(lane_base + 32 * c, r);
+                    if (tok >= 0) {
+#pragma unroll
+                        for (int q = 0; q < 8; q++)
+                            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                                         ::"l"(dst + 32 * c + 4 * q), "f"(coef * __uint_as_float(r[4 * q])),
+                                           "f"(coef * __uint_as_float(r[4 * q + 1])),
+                                           "f"(coef * __uint_as_float(r[4 * q + 2])),
+                                           "f"(coef * __uint_as_float(r[4 * q + 3]))
+                                         : "memory");
                     }
                 }
             }
-        } else {
-            const int n0 = nt * 128;
-            float coef = 0.0f;
-            float* dst = nullptr;
-            if (tok >= 0) {
-                const int j = g.ws.perm_rank[row];
-                coef = g.w[tok * g.k + j] * ts[2];
-                dst = g.y + (size_t)tok * g.H + n0;
-            }
-#pragma unroll
-            for (int c = 0; c < 4; c++) {
-                uint32_t r[32];
-                tmem_ld_32x32(lane_base + 32 * c, r);
-                if (tok >= 0) {
-#pragma unroll
-                    for (int q = 0; q < 8; q++)
-                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
-                                     ::"l"(dst + 32 * c + 4 * q), "f"(coef * __uint_as_float(r[4 * q])),
-                                       "f"(coef * __uint_as_float(r[4 * q + 1])), "f"(coef * __uint_as_float(r[4 * q + 2])),
-                                       "f"(coef * __uint_as_float(r[4 * q + 3]))
-                                     : "memory");
-                }
-            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[a]);
         }
-        tc_fence_before();
     }
     __syncthreads();
     if (warp == 1) {
@@ -544,7 +592,8 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
         attr = true;
     }
     g.NT = c.I / 64;
-    grouped_gemm_kernel<1><<<PL.MT * g.NT, kPThreads, smem, s>>>(ma1, msa1, mb1, msb1, g);
+    const int grid1 = std::min(PL.MT * g.NT, p->num_sms);
+    grouped_gemm_kernel<1><<<grid1, kPThreads, smem, s>>>(ma1, msa1, mb1, msb1, g);
     MOE_CUDA_TRY(cudaGetLastError());
     // GEMM2 reads the down rows of the slot with its own pitch
     g.b_rows_per_slot = B.bytes / dr;
@@ -552,7 +601,8 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
     g.d_row = B.off[4] / dr;
     g.d_sf_row = B.off[5] / ds;
     g.NT = c.H / 128;
-    grouped_gemm_kernel<2><<<PL.MT * g.NT, kPThreads, smem, s>>>(ma2, msa2, mb2, msb2, g);
+    const int grid2 = std::min(PL.MT * g.NT, p->num_sms);
+    grouped_gemm_kernel<2><<<grid2, kPThreads, smem, s>>>(ma2, msa2, mb2, msb2, g);
     MOE_CUDA_TRY(cudaGetLastError());
     return MOE_OK;
 }

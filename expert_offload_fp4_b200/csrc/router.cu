@@ -26,6 +26,7 @@ router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr,
     extern __shared__ float xs[];  // [TT][H] fp32
     __shared__ int s_last;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_trigger();   // the slot lookup may launch now; it waits for this grid to finish
     const int t0 = blockIdx.y * TT;
     const int nt = min(TT, T - t0);
 
