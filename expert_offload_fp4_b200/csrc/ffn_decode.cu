@@ -344,6 +344,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
     }
     // ---- the slot lookup's outputs (slot_of, tickets) are needed from here on
     pdl_wait();
+    if (trace && tid == 0) trace[1] = globaltimer();
     // ---- prologue: barriers, groups, activations (parallel; the stage ring is
     // still unused, so its first bytes hold the per-(token, rank) scratch)
     int* e_s = reinterpret_cast<int*>(stages);            // [n] expert or -1

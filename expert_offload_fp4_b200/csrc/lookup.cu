@@ -234,12 +234,12 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(LookupArgs a) {
     for (int i = tid; i < a.n; i += blockDim.x) a.slot_of[i] = uslot[umap[a.idx[i]]];
     __syncthreads();
     if (tid == 0) {
+        // the host reads the record after the kernel's completion event, which
+        // makes these mapped-memory writes visible
         a.out->n_uniq = nu;
         a.out->n_miss = nm;
         a.out->status = 0;
-        __threadfence_system();
         a.out->seq = a.seq;
-        __threadfence_system();
     }
 }
 

@@ -30,10 +30,16 @@ router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr,
     const int t0 = blockIdx.y * TT;
     const int nt = min(TT, T - t0);
 
-    for (int i = threadIdx.x; i < TT * H; i += blockDim.x) {
-        const int t = i / H;
-        const uint32_t b = t < nt ? x[size_t(t0 + t) * H + (i - t * H)] : 0;
-        xs[i] = __uint_as_float(b << 16);
+    for (int v = threadIdx.x; v < TT * H / 8; v += blockDim.x) {
+        const int t = (v * 8) / H, h = v * 8 - t * H;
+        uint4 q = make_uint4(0, 0, 0, 0);
+        if (t < nt) q = *reinterpret_cast<const uint4*>(x + size_t(t0 + t) * H + h);
+        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+        float4* dst = reinterpret_cast<float4*>(xs + t * H + h);
+        dst[0] = make_float4(__uint_as_float(u[0] << 16), __uint_as_float(u[0] & 0xFFFF0000u),
+                             __uint_as_float(u[1] << 16), __uint_as_float(u[1] & 0xFFFF0000u));
+        dst[1] = make_float4(__uint_as_float(u[2] << 16), __uint_as_float(u[2] & 0xFFFF0000u),
+                             __uint_as_float(u[3] << 16), __uint_as_float(u[3] & 0xFFFF0000u));
     }
     __syncthreads();
 
@@ -44,30 +50,45 @@ router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr,
 #pragma unroll
         for (int t = 0; t < TT; t++) acc[a][t] = 0.0f;
 
-    const int nchunk = H / 8;
-    for (int c = lane; c < nchunk; c += 32) {
-        float wf[EPW][8];
+    // H % 256 == 0, so every lane owns exactly H / 256 chunks: c = lane + 32 q.
+    // They are taken kPre at a time, all loads of a batch issued before any use.
+    const int nper = H / 256;
+    constexpr int kPre = EPW == 1 ? 8 : 4;
+    for (int q0 = 0; q0 < nper; q0 += kPre) {
+        uint4 pre[EPW][kPre];
 #pragma unroll
-        for (int a = 0; a < EPW; a++) {
-            const int e = e0 + a;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (e < E) v = __ldg(reinterpret_cast<const uint4*>(wr + size_t(e) * H) + c);
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        for (int a = 0; a < EPW; a++)
 #pragma unroll
-            for (int q = 0; q < 4; q++) {
-                wf[a][2 * q] = __uint_as_float(u[q] << 16);
-                wf[a][2 * q + 1] = __uint_as_float(u[q] & 0xFFFF0000u);
+            for (int q = 0; q < kPre; q++) {
+                const int e = e0 + a;
+                pre[a][q] = (q0 + q < nper && e < E)
+                                ? __ldg(reinterpret_cast<const uint4*>(wr + size_t(e) * H) + lane + 32 * (q0 + q))
+                                : make_uint4(0, 0, 0, 0);
             }
-        }
 #pragma unroll
-        for (int t = 0; t < TT; t++) {
-            const float4 xa = *reinterpret_cast<const float4*>(xs + t * H + c * 8);
-            const float4 xb = *reinterpret_cast<const float4*>(xs + t * H + c * 8 + 4);
-            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        for (int q = 0; q < kPre; q++) {
+            if (q0 + q >= nper) break;
+            const int c = lane + 32 * (q0 + q);
+            float wf[EPW][8];
 #pragma unroll
-            for (int a = 0; a < EPW; a++)
+            for (int a = 0; a < EPW; a++) {
+                const uint32_t u[4] = {pre[a][q].x, pre[a][q].y, pre[a][q].z, pre[a][q].w};
 #pragma unroll
-                for (int q = 0; q < 8; q++) acc[a][t] = fmaf(xv[q], wf[a][q], acc[a][t]);
+                for (int r = 0; r < 4; r++) {
+                    wf[a][2 * r] = __uint_as_float(u[r] << 16);
+                    wf[a][2 * r + 1] = __uint_as_float(u[r] & 0xFFFF0000u);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < TT; t++) {
+                const float4 xa = *reinterpret_cast<const float4*>(xs + t * H + c * 8);
+                const float4 xb = *reinterpret_cast<const float4*>(xs + t * H + c * 8 + 4);
+                const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                for (int a = 0; a < EPW; a++)
+#pragma unroll
+                    for (int r = 0; r < 8; r++) acc[a][t] = fmaf(xv[r], wf[a][r], acc[a][t]);
+            }
         }
     }
 #pragma unroll
@@ -177,6 +198,8 @@ int route_impl(const void* x_bf16, const void* wr_bf16, const float* bias, int T
     if (!x_bf16 || !wr_bf16 || !idx || !w || !logits || !cnt) return fail(MOE_EINVAL, "null pointer");
     if (T <= 0 || H <= 0 || H % 256 || E <= 0 || E > kMaxE || k <= 0 || k > kMaxK || k > E)
         return fail(MOE_EINVAL, "route: need T > 0, H % 256 == 0, 0 < k <= min(E, 32), E <= 1024");
+    if ((reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(wr_bf16)) & 15)
+        return fail(MOE_EINVAL, "route: x and W_r must be 16-byte aligned");
     if (size_t(kRouterTileMax) * H * sizeof(float) > 200 * 1024)
         return fail(MOE_EINVAL, "route: H too large for the shared-memory x tile");
     const uint16_t* x = (const uint16_t*)x_bf16;

@@ -156,7 +156,8 @@ int moe_pool_slot_ptr(moe_pool* pool, int slot, void** ptr, size_t* bytes);
  * and w [T,k] fp32 in rank order.  workspace: device scratch of
  * moe_route_workspace_bytes(T, E) bytes, its counters zero before the first
  * use (the call leaves them zero).  Limits: H % 256 == 0, E <= 1024,
- * k <= min(E, 32).  Errors: MOE_EINVAL. */
+ * k <= min(E, 32), x and W_r 16-byte aligned (both are read 16 bytes at a
+ * time).  Errors: MOE_EINVAL. */
 size_t moe_route_workspace_bytes(int T, int E);
 int moe_route(const void* x_bf16, const void* wr_bf16, const float* bias, int T, int H, int E,
               int k, int renormalize, int32_t* idx, float* w, void* workspace,
@@ -229,7 +230,8 @@ int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
 
 /* Tracing: when buf is a device buffer of at least 8 * 148 (8 per SM) u64,
  * each CTA of every later moe_expert_ffn launch writes global-timer stamps (ns)
- * of its phases: [0] start, [1] expert table built, [2] activations staged,
+ * of its phases: [0] start, [1] the preceding kernel (the slot lookup)
+ * complete and the activations staged, [2] expert table built,
  * [3] first item's weights landed, [4] gate/up items done and published,
  * [5] first down item's h dependency met, [6] last item done, [7] end.
  * Unwritten entries keep their old value.  NULL turns tracing off. */

@@ -87,5 +87,8 @@ def test_route_argument_checks_need_no_gpu(lib):
     assert L.moe_route(p, p, None, 4, 256, 16, 17, 1, p, p, p, ws, None) == lib.MOE_EINVAL
     assert L.moe_route(p, p, None, 4, 256, 16, 2, 1, p, p, p, 8, None) == lib.MOE_EINVAL
     assert b"workspace" in L.moe_last_error()
+    odd = C.c_void_p(p.value | 1)   # x and W_r are read 16 bytes at a time
+    assert L.moe_route(odd, p, None, 4, 256, 16, 2, 1, p, p, p, ws, None) == lib.MOE_EINVAL
+    assert b"aligned" in L.moe_last_error()
     assert L.moe_combine(p, 4, 2, 254, p, None) == lib.MOE_EINVAL
     assert L.moe_set_wait_limits(-1.0, 1.0, 1.0) == lib.MOE_EINVAL
