@@ -244,7 +244,8 @@ def decode_run(torch, m, w, pool, T, xs_dev, wr, bias, steps, warmup, events=Fal
     torch.cuda.synchronize()
     st0 = pool.stats()
     if events:
-        lo.ffn_events, lo.copy_events = [], []
+        lo.copy_events = []
+        lo.reserve_copy_events(steps * w.L)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(cur)
     for s in range(steps):
@@ -257,7 +258,6 @@ def decode_run(torch, m, w, pool, T, xs_dev, wr, bias, steps, warmup, events=Fal
     d = {k: st1[k] - st0[k] for k in st1}
     out = dict(ms=ms, stats=d, status=int(lo.status.item()))
     if events:
-        out["ffn"] = [(a.elapsed_time(b), u, mm) for (a, b), u, mm in lo.ffn_events]
         out["copy"] = [(a.elapsed_time(b), n) for (a, b), n in lo.copy_events]
     return out
 
@@ -334,13 +334,15 @@ def ffn_only(args, w, T):
     ms, uniq = ffn_roofline(torch, m, wl, pool, T, x_dev, wr, bias, reps=2)
     phases = None
     if args.trace:
-        buf = torch.zeros((148, 8), dtype=torch.int64, device="cuda")
+        buf = torch.zeros((148, 64), dtype=torch.int64, device="cuda")
         m._lib.load().moe_set_ffn_trace(buf.data_ptr())
         ffn_roofline(torch, m, wl, pool, T, x_dev, wr, bias, reps=1)
         m._lib.load().moe_set_ffn_trace(None)
         tr = buf.cpu().numpy().astype(np.float64)
         t0 = tr[:, 0].min()
-        rel = (tr - t0) / 1000.0
+        rel = (tr[:, :8] - t0) / 1000.0
+        if args.trace_out:
+            np.save(args.trace_out, buf.cpu().numpy())
         phases = {name: [round(float(np.median(rel[:, i])), 2), round(float(rel[:, i].max()), 2)]
                   for i, name in enumerate(["start", "lookup_done", "table", "first_data", "a_done",
                                             "b_dep", "items_done", "end"])}
@@ -493,6 +495,7 @@ def main():
                          "(a few layers), e.g. for an ncu capture")
     ap.add_argument("--layers", type=int, default=4, help="layer positions in --mode ffn")
     ap.add_argument("--trace", action="store_true", help="--mode ffn: per-CTA phase timestamps")
+    ap.add_argument("--trace-out", default="", help="--trace: also save the raw stamps (.npy)")
     ap.add_argument("--host-layers", type=int, default=8,
                     help="--mode offload: distinct host copies of the 40 layers (pinned RAM)")
     ap.add_argument("--no-overlap", action="store_true",

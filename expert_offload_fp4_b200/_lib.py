@@ -70,6 +70,8 @@ SIGNATURES = {
     "moe_stream_misses": (i32, [vp, i32, C.POINTER(Miss), i32, vp]),
     "moe_expert_ffn": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp]),
     "moe_combine": (i32, [vp, i32, i32, i32, vp, vp]),
+    "moe_decode_layer": (i32, [vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,
+                               C.POINTER(LookupResult), vp, vp, i32, vp, vp]),
     "qstar_split": (i32, [i32, f64, f64, C.POINTER(i32), C.POINTER(i32), C.POINTER(f64)]),
     "moe_dequant_slot": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_set_wait_limits": (i32, [f64, f64, f64]),

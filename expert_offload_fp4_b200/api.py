@@ -173,6 +173,20 @@ def expert_ffn(pool, layer, x, idx, w, slot_of, y_part, status, stream=None):
         _s(stream)))
 
 
+def decode_layer(pool, layer, x, wr, bias, renormalize, idx, w, slot_of, y_part, y, status, ws,
+                 lookup=None, copy_events=None, overlap=True, stream=None, copy_stream=None):
+    """moe_decode_layer: route, lookup, FFN, miss copies and combine of one layer."""
+    T = x.shape[0]
+    cs = copy_stream if copy_stream is not None else stream
+    ev0, ev1 = (None, None) if copy_events is None else (C.c_void_p(copy_events[0].cuda_event),
+                                                        C.c_void_p(copy_events[1].cuda_event))
+    L.check("moe_decode_layer", pool.lib.moe_decode_layer(
+        pool.handle, int(layer), _p(x), T, _p(wr), _p(bias), int(renormalize), _p(idx), _p(w),
+        _p(slot_of), _p(y_part), _p(y), _p(status), _p(ws), ws.numel(),
+        C.byref(lookup.res) if lookup is not None else None, ev0, ev1, 1 if overlap else 0,
+        _s(stream), _s(cs)))
+
+
 def combine(y_part, y, stream=None):
     T, k, H = y_part.shape
     L.check("moe_combine", L.load().moe_combine(_p(y_part), T, k, H, _p(y), _s(stream)))

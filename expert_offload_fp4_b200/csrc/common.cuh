@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <utility>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -185,6 +186,25 @@ __device__ __forceinline__ void red_release_add(unsigned int* p, unsigned int v)
 // visible (both are no-ops for kernels launched without the attribute).
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Host: launch `kern` with programmatic stream serialisation, so that it may
+// start while the previous kernel of the stream runs (the kernel must
+// pdl_wait() before it touches anything that kernel writes or reads).
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                     cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
+}
 
 // Named barrier over `nthreads` threads (a multiple of 32) with id `id` (1..15).
 __device__ __forceinline__ void named_sync(int id, int nthreads) {

@@ -32,6 +32,7 @@ constexpr int kDoneIdx = kMaxDecodePairs + 1;
 
 struct Group {
     int expert, slot, M, pos;
+    int ready;                 // the slot already showed the ticket this call needs
     float ts[3];
     float wt[kMaxDecodeT];     // routing weight of each member (token, rank)
     uint8_t tok[kMaxDecodeT];
@@ -57,30 +58,10 @@ struct FfnArgs {
     int T, k, H, I, E, S, layer, fmt;
     int RA, RB, stage_bytes, nstage;
     unsigned long long ready_ns, dep_ns, pipe_ns;
-    unsigned long long* trace;   // optional [gridDim][8] phase timestamps (ns), or null
+    unsigned long long* trace;   // optional [gridDim][64] phase timestamps (ns), or null
 };
 
 // ------------------------------------------------------------------ helpers
-
-// 16 code bytes = 32 E2M1 elements -> 16 f16x2 words (word i = elements 2i, 2i+1)
-__device__ __forceinline__ void decode_e2m1_16B(const uint4 c, uint32_t (&w)[16]) {
-    const uint32_t v[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-    for (int q = 0; q < 4; q++)
-        asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;"
-            " cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;"
-            " cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
-            : "=r"(w[4 * q]), "=r"(w[4 * q + 1]), "=r"(w[4 * q + 2]), "=r"(w[4 * q + 3])
-            : "r"(v[q]));
-}
-
-// acc += w.lo * x.lo + w.hi * x.hi, products exact, fp32 accumulation
-__device__ __forceinline__ float fma_f16x2(uint32_t w, uint32_t x, float acc) {
-    asm("{ .reg .f16 wl, wh, xl, xh; mov.b32 {wl, wh}, %1; mov.b32 {xl, xh}, %2;"
-        " fma.rn.f32.f16 %0, wl, xl, %0; fma.rn.f32.f16 %0, wh, xh, %0; }"
-        : "+f"(acc) : "r"(w), "r"(x));
-    return acc;
-}
 
 __device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
     return e == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23);
@@ -110,27 +91,39 @@ __device__ __forceinline__ float act_scale(float amax) {
 // of chunk c (16 code bytes) are four 16-byte pieces, piece q of chunk c at
 // uint4 index q*cpr + c (cpr = chunks per row), so lanes reading consecutive
 // chunks touch consecutive 16-byte words (no bank conflicts).  Inside a piece
-// the 8 elements are ordered 0,4,1,5,2,6,3,7: f16x2 word i holds elements
-// (i, i+4), the pairing the E2M1 decode below produces.
+// the 8 elements are ordered 0,4,2,6,1,5,3,7: the f16x2 words hold the element
+// pairs (0,4), (2,6), (1,5), (3,7), the pairing the E2M1 decode below produces.
 __device__ __forceinline__ int act_index(int h, int cpr) {
     const int c = h >> 5, o = h & 31, e = o & 7;
-    return (((o >> 3) * cpr + c) << 3) + (e < 4 ? 2 * e : 2 * (e - 4) + 1);
+    return (((o >> 3) * cpr + c) << 3) + (((e & 1) << 2) | (e & 2) | (e >> 2));
+}
+
+// Eight values of one piece (elements 0..7) as the four f16x2 words of that order.
+__device__ __forceinline__ uint4 pack_piece(const float (&f)[8]) {
+    const __half2 w0 = __floats2half2_rn(f[0], f[4]), w1 = __floats2half2_rn(f[2], f[6]);
+    const __half2 w2 = __floats2half2_rn(f[1], f[5]), w3 = __floats2half2_rn(f[3], f[7]);
+    return make_uint4(*reinterpret_cast<const uint32_t*>(&w0), *reinterpret_cast<const uint32_t*>(&w1),
+                      *reinterpret_cast<const uint32_t*>(&w2), *reinterpret_cast<const uint32_t*>(&w3));
 }
 
 // 32 E2M1 codes (16 bytes; element n of a 32-bit word in bits 4n..4n+3) to 16
-// f16x2 words, each holding e2m1 * 2^-14 exactly: the code's magnitude bits go
-// to f16 bits 11..9 (exponent low bits + top mantissa bit) and its sign to bit
-// 15, so 2^-14 scales every value, the E2M1 subnormal 0.5 included.  Word 4q+i
-// holds elements (8q+i, 8q+i+4) of the chunk: one shift serves both halves.
+// f16x2 words, each value e2m1 * 2^-14 exactly: a code's magnitude bits go to
+// f16 bits 11..9 (exponent low bits and the top mantissa bit) and its sign to
+// bit 15, so 2^-14 scales every value, the E2M1 subnormal 0.5 included.  Per
+// 32-bit word the f16 high bytes of the even elements (low nibbles) and of the
+// odd elements (high nibbles) are formed in place, four bytes at a time; byte
+// moves then give the words (e0,e4), (e2,e6), (e1,e5), (e3,e7).
 __device__ __forceinline__ void decode_e2m1_x2(const uint4 c, uint32_t (&w)[16]) {
     const uint32_t v[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int q = 0; q < 4; q++) {
         const uint32_t x = v[q];
-        w[4 * q + 0] = ((x << 9) & 0x0E000E00u) | ((x << 12) & 0x80008000u);
-        w[4 * q + 1] = ((x << 5) & 0x0E000E00u) | ((x << 8) & 0x80008000u);
-        w[4 * q + 2] = ((x << 1) & 0x0E000E00u) | ((x << 4) & 0x80008000u);
-        w[4 * q + 3] = ((x >> 3) & 0x0E000E00u) | (x & 0x80008000u);
+        const uint32_t ev = ((x << 1) & 0x0E0E0E0Eu) | ((x << 4) & 0x80808080u);   // bytes: e0 e2 e4 e6
+        const uint32_t od = ((x >> 3) & 0x0E0E0E0Eu) | (x & 0x80808080u);          // bytes: e1 e3 e5 e7
+        w[4 * q + 0] = __byte_perm(ev, 0u, 0x2404);
+        w[4 * q + 1] = ev & 0xFF00FF00u;
+        w[4 * q + 2] = __byte_perm(od, 0u, 0x2404);
+        w[4 * q + 3] = od & 0xFF00FF00u;
     }
 }
 
@@ -140,10 +133,32 @@ __device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c
     return d;
 }
 
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// acc + (v.lo + v.hi) * s, with s an f16 (an E4M3 scale is exact in f16): two
+// mixed fmas, each product exact, each sum rounded once to fp32.
+__device__ __forceinline__ float fma2_f16(uint32_t v, uint16_t s, float acc) {
+    asm("{ .reg .f16 lo, hi, sc; mov.b32 {lo, hi}, %1; mov.b16 sc, %2;"
+        " fma.rn.f32.f16 %0, lo, sc, %0; fma.rn.f32.f16 %0, hi, sc, %0; }"
+        : "+f"(acc) : "r"(v), "h"(s));
+    return acc;
+}
+
 __device__ __forceinline__ float f16x2_sum(uint32_t v) {
     const __half2 h = *reinterpret_cast<const __half2*>(&v);
     const float2 f = __half22float2(h);
     return f.x + f.y;
+}
+
+// two E4M3 bytes (lo = first block) -> two f16 scales in one word
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    uint32_t h2;
+    asm("{ .reg .b16 lo; cvt.u16.u32 lo, %1; cvt.rn.f16x2.e4m3x2 %0, lo; }" : "=r"(h2) : "r"(two));
+    return h2;
 }
 
 // Dot products of one row chunk (16 code bytes = 32 elements) with MT activation
@@ -155,16 +170,10 @@ __device__ __forceinline__ void chunk_dot(const uint8_t* code, const uint8_t* sc
                                           const __half* const* act, int M, float (&acc)[MT]) {
     uint32_t wv[16];
     decode_e2m1_x2(*reinterpret_cast<const uint4*>(code + 16 * c), wv);
-    float s0, s1;
-    if (FMT == MOE_NVFP4) {
-        const uint32_t two = (uint32_t)scl[2 * c] | ((uint32_t)scl[2 * c + 1] << 8);
-        const float2 s = e4m3x2_to_f32(two);
-        s0 = s.x;
-        s1 = s.y;
-    } else {
-        s0 = e8m0_to_f32(scl[c]);
-        s1 = s0;
-    }
+    uint32_t s2 = 0u;
+    float sm = 0.0f;
+    if (FMT == MOE_NVFP4) s2 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(scl + 2 * c));
+    else sm = e8m0_to_f32(scl[c]);
 #pragma unroll
     for (int m = 0; m < MT; m++) {
         if (m >= M) break;
@@ -172,7 +181,7 @@ __device__ __forceinline__ void chunk_dot(const uint8_t* code, const uint8_t* sc
         const uint4 x0 = xp[0], x1 = xp[cpr], x2 = xp[2 * cpr], x3 = xp[3 * cpr];
         const uint32_t xv[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
                                  x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
-        uint32_t pa = 0u, pb = 0u, pc = 0u, pd = 0u;   // two chains per block
+        uint32_t pa = 0u, pb = 0u, pc = 0u, pd = 0u;   // two chains per 16-element block
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
             pa = hfma2_u32(wv[i], xv[i], pa);
@@ -181,10 +190,10 @@ __device__ __forceinline__ void chunk_dot(const uint8_t* code, const uint8_t* sc
             pd = hfma2_u32(wv[9 + i], xv[9 + i], pd);
         }
         if (FMT == MOE_NVFP4) {
-            acc[m] = fmaf(f16x2_sum(pa) + f16x2_sum(pb), s0, acc[m]);
-            acc[m] = fmaf(f16x2_sum(pc) + f16x2_sum(pd), s1, acc[m]);
+            acc[m] = fma2_f16(hadd2_u32(pa, pb), (uint16_t)(s2 & 0xFFFFu), acc[m]);
+            acc[m] = fma2_f16(hadd2_u32(pc, pd), (uint16_t)(s2 >> 16), acc[m]);
         } else {
-            acc[m] = fmaf((f16x2_sum(pa) + f16x2_sum(pb)) + (f16x2_sum(pc) + f16x2_sum(pd)), s0, acc[m]);
+            acc[m] = fmaf(f16x2_sum(hadd2_u32(hadd2_u32(pa, pb), hadd2_u32(pc, pd))), sm, acc[m]);
         }
     }
 }
@@ -198,14 +207,14 @@ __device__ __forceinline__ void chunk_dot_pair(const uint8_t* gcode, const uint8
     uint32_t wg[16], wu[16];
     decode_e2m1_x2(*reinterpret_cast<const uint4*>(gcode + 16 * c), wg);
     decode_e2m1_x2(*reinterpret_cast<const uint4*>(ucode + 16 * c), wu);
-    float g0, g1, u0, u1;
+    uint32_t sg2 = 0u, su2 = 0u;
+    float sgm = 0.0f, sum_ = 0.0f;
     if (FMT == MOE_NVFP4) {
-        const float2 sg = e4m3x2_to_f32((uint32_t)gscl[2 * c] | ((uint32_t)gscl[2 * c + 1] << 8));
-        const float2 su = e4m3x2_to_f32((uint32_t)uscl[2 * c] | ((uint32_t)uscl[2 * c + 1] << 8));
-        g0 = sg.x; g1 = sg.y; u0 = su.x; u1 = su.y;
+        sg2 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(gscl + 2 * c));
+        su2 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(uscl + 2 * c));
     } else {
-        g0 = g1 = e8m0_to_f32(gscl[c]);
-        u0 = u1 = e8m0_to_f32(uscl[c]);
+        sgm = e8m0_to_f32(gscl[c]);
+        sum_ = e8m0_to_f32(uscl[c]);
     }
 #pragma unroll
     for (int m = 0; m < MT; m++) {
@@ -227,13 +236,13 @@ __device__ __forceinline__ void chunk_dot_pair(const uint8_t* gcode, const uint8
             ud = hfma2_u32(wu[9 + i], xv[9 + i], ud);
         }
         if (FMT == MOE_NVFP4) {
-            ag[m] = fmaf(f16x2_sum(ga) + f16x2_sum(gb), g0, ag[m]);
-            ag[m] = fmaf(f16x2_sum(gc) + f16x2_sum(gd), g1, ag[m]);
-            au[m] = fmaf(f16x2_sum(ua) + f16x2_sum(ub), u0, au[m]);
-            au[m] = fmaf(f16x2_sum(uc) + f16x2_sum(ud), u1, au[m]);
+            ag[m] = fma2_f16(hadd2_u32(ga, gb), (uint16_t)(sg2 & 0xFFFFu), ag[m]);
+            ag[m] = fma2_f16(hadd2_u32(gc, gd), (uint16_t)(sg2 >> 16), ag[m]);
+            au[m] = fma2_f16(hadd2_u32(ua, ub), (uint16_t)(su2 & 0xFFFFu), au[m]);
+            au[m] = fma2_f16(hadd2_u32(uc, ud), (uint16_t)(su2 >> 16), au[m]);
         } else {
-            ag[m] = fmaf((f16x2_sum(ga) + f16x2_sum(gb)) + (f16x2_sum(gc) + f16x2_sum(gd)), g0, ag[m]);
-            au[m] = fmaf((f16x2_sum(ua) + f16x2_sum(ub)) + (f16x2_sum(uc) + f16x2_sum(ud)), u0, au[m]);
+            ag[m] = fmaf(f16x2_sum(hadd2_u32(hadd2_u32(ga, gb), hadd2_u32(gc, gd))), sgm, ag[m]);
+            au[m] = fmaf(f16x2_sum(hadd2_u32(hadd2_u32(ua, ub), hadd2_u32(uc, ud))), sum_, au[m]);
         }
     }
 }
@@ -294,7 +303,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     volatile unsigned int* abort_flag = a.ctr + kAbortIdx;
-    unsigned long long* trace = a.trace ? a.trace + (size_t)blockIdx.x * 8 : nullptr;
+    unsigned long long* trace = a.trace ? a.trace + (size_t)blockIdx.x * 64 : nullptr;
     if (trace && tid == 0) trace[0] = globaltimer();
     const int bs = FMT == MOE_MXFP4 ? 32 : 16;
     const unsigned long long codeA = (unsigned long long)a.H / 2, sclA = (unsigned long long)a.H / bs;
@@ -331,19 +340,13 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                 f[2 * i] = __uint_as_float(u[i] << 16) * sc;
                 f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u) * sc;
             }
-            // one piece: f16x2 words (0,4), (1,5), (2,6), (3,7)
-            uint32_t o[4];
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const __half2 h2 = __floats2half2_rn(f[i], f[i + 4]);
-                o[i] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            *reinterpret_cast<uint4*>(xs + t * a.H + act_index(h, cprA)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(xs + t * a.H + act_index(h, cprA)) = pack_piece(f);
             if (h == 0) xinv[t] = 1.0f / sc;
         }
     }
     // ---- the slot lookup's outputs (slot_of, tickets) are needed from here on
     pdl_wait();
+    pdl_trigger();   // the combine may launch; it waits for this grid to finish
     if (trace && tid == 0) trace[1] = globaltimer();
     // ---- prologue: barriers, groups, activations (parallel; the stage ring is
     // still unused, so its first bytes hold the per-(token, rank) scratch)
@@ -353,6 +356,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
     int* lead_s = reinterpret_cast<int*>(need_s + kMaxDecodePairs);   // first entry of my expert
     int* mi_s = lead_s + kMaxDecodePairs;                  // my index inside the group
     int* grank_s = mi_s + kMaxDecodePairs;                 // group rank of a leader
+    int* rdy_s = grank_s + kMaxDecodePairs;                // slot shows the needed ticket
+    float* ts_s = reinterpret_cast<float*>(rdy_s + kMaxDecodePairs);   // [n][3] tensor scales
     const int n = a.T * a.k;
     if (tid == 0) {
         for (int i = 0; i < a.nstage; i++) {
@@ -363,13 +368,28 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
     }
     __syncthreads();   // activation staging above used hinv; the table below uses the stage ring
     if (tid < n) {
+        // one dependent round of loads: the slot's tickets and the tensor scales
         const int e = a.idx[tid], sl = a.slot_of[tid];
         int bad = 0;
         if (e < 0 || e >= a.E) bad |= MOE_STATUS_BAD_EXPERT;
         if (sl < 0 || sl >= a.S) bad |= MOE_STATUS_BAD_SLOT;
+        uint32_t nd = 0u, rd = 1u;
+        float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f;
+        if (!bad) {
+            nd = a.need[sl];
+            rd = ld_acquire_sys_u32(a.ready + sl);
+            const float* ts = a.tscale + ((size_t)a.layer * a.E + e) * 3;
+            t0 = ts[0];
+            t1 = ts[1];
+            t2 = ts[2];
+        }
         e_s[tid] = bad ? -1 : e;
         s_s[tid] = sl;
-        need_s[tid] = bad ? 0u : a.need[sl];
+        need_s[tid] = nd;
+        rdy_s[tid] = (rd == nd);
+        ts_s[3 * tid] = t0;
+        ts_s[3 * tid + 1] = t1;
+        ts_s[3 * tid + 2] = t2;
         if (bad && blockIdx.x == 0) atomicOr(a.status, bad);
     }
     __syncthreads();
@@ -405,10 +425,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
         G.slot = s_s[tid];
         G.M = M;
         G.pos = pos;
-        const float* ts = a.tscale + ((size_t)a.layer * a.E + e) * 3;
-        G.ts[0] = ts[0];
-        G.ts[1] = ts[1];
-        G.ts[2] = ts[2];
+        G.ready = rdy_s[tid];
+        G.ts[0] = ts_s[3 * tid];
+        G.ts[1] = ts_s[3 * tid + 1];
+        G.ts[2] = ts_s[3 * tid + 2];
     }
     __syncthreads();
     if (tid < n && e_s[tid] >= 0) {
@@ -487,21 +507,14 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
     if (warp == kNC) {
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
-            // one sweep over the groups this CTA touches: experts already resident
-            // (or landed) are marked ready behind a single proxy fence; the others are
-            // waited for when their first item comes up
+            // experts whose slot showed the needed ticket when the table was built
+            // (acquired there, ordered before this thread by the block barrier) are
+            // read behind one proxy fence; the others are waited for when their
+            // first item comes up
             uint32_t ready_mask[kMaxDecodePairs / 32] = {0, 0, 0, 0};
-            int any = 0;
-            for (int j = 0; j < nmine; j++) {
-                const int item = item_of(j);
-                const int g = item >= NA ? (item - NA) / nB_per : item / nA_per;
-                if (ready_mask[g >> 5] & (1u << (g & 31))) continue;
-                if (ld_acquire_u32(a.ready + groups[g].slot) == a.need[groups[g].slot]) {
-                    ready_mask[g >> 5] |= 1u << (g & 31);
-                    any = 1;
-                }
-            }
-            if (any) fence_proxy_async_global();
+            for (int g = 0; g < ng; g++)
+                if (groups[g].ready) ready_mask[g >> 5] |= 1u << (g & 31);
+            fence_proxy_async_global();
             for (int j = 0; j < nmine; j++) {
                 const int item = item_of(j);
                 const int st = j % a.nstage, round = j / a.nstage;
@@ -523,6 +536,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                 int nsrc = 0;
                 const StageMap m = stage_map(item, src, len, nsrc);
                 uint8_t* dst = stages + (size_t)st * a.stage_bytes;
+                if (trace && j < 16) trace[40 + j] = globaltimer();
                 mbar_arrive_expect_tx(&full[st], m.bytes);
                 uint32_t o = 0;
                 for (int i = 0; i < nsrc; i++) {
@@ -558,6 +572,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                 *abort_flag = 1;
             }
             if (trace && tid == 0 && j == 0) trace[3] = globaltimer();
+            if (trace && tid == 0 && j < 16) trace[8 + 2 * j] = globaltimer();
             unsigned long long src[4];
             uint32_t len[4];
             int nsrc;
@@ -640,15 +655,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                         const float4* hrow = reinterpret_cast<const float4*>(a.hbuf + (size_t)(G.pos + q) * a.I);
                         for (int v = lane; v < a.I / 8; v += 32) {
                             const float4 f0 = __ldcg(hrow + 2 * v), f1 = __ldcg(hrow + 2 * v + 1);
-                            const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-                            uint32_t o[4];
-#pragma unroll
-                            for (int i = 0; i < 4; i++) {
-                                const __half2 h2 = __floats2half2_rn(f[i] * sc, f[i + 4] * sc);
-                                o[i] = *reinterpret_cast<const uint32_t*>(&h2);
-                            }
-                            *reinterpret_cast<uint4*>(hs + (size_t)q * a.I + act_index(8 * v, cprB)) =
-                                make_uint4(o[0], o[1], o[2], o[3]);
+                            const float f[8] = {f0.x * sc, f0.y * sc, f0.z * sc, f0.w * sc,
+                                                f1.x * sc, f1.y * sc, f1.z * sc, f1.w * sc};
+                            *reinterpret_cast<uint4*>(hs + (size_t)q * a.I + act_index(8 * v, cprB)) = pack_piece(f);
                         }
                     }
                     named_sync(1, kNC * 32);
@@ -685,6 +694,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
+            if (trace && tid == 0 && j < 16) trace[9 + 2 * j] = globaltimer();
         }
         publish();
         if (trace && tid == 0) trace[6] = globaltimer();
@@ -692,7 +702,11 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
 
     // ---- epilogue: the last CTA clears the per-call counters
     __syncthreads();
-    if (trace && tid == 0) trace[7] = globaltimer();
+    if (trace && tid == 0) {
+        trace[7] = globaltimer();
+        trace[56] = (unsigned long long)nmine;
+        trace[57] = (unsigned long long)(a1 - a0);
+    }
     if (tid == 0) {
         __threadfence();
         const unsigned int prev = atomicAdd(a.ctr + kDoneIdx, 1u);
@@ -710,6 +724,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
 // ------------------------------------------------------------------ combine
 
 __global__ void combine_kernel(const float* __restrict__ y_part, int T, int k, int H, uint16_t* __restrict__ y) {
+    pdl_wait();      // y_part comes from the expert FFN
+    pdl_trigger();   // the next layer's router may launch and fetch its weights
     const size_t n4 = (size_t)T * H / 4;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         const size_t e = i * 4;
@@ -787,6 +803,9 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     const size_t budget = 227 * 1024;
     if (fixed + 2 * (size_t)a.stage_bytes > budget) return fail(MOE_EINVAL, "decode FFN: shapes exceed shared memory");
     a.nstage = (int)std::min<size_t>(12, (budget - fixed) / a.stage_bytes);
+    // the prologue keeps its per-(token, rank) table (7 ints + 3 floats each) in the ring
+    if ((size_t)a.nstage * a.stage_bytes < 10 * 4 * (size_t)kMaxDecodePairs)
+        return fail(MOE_EINVAL, "decode FFN: stage ring smaller than the prologue table");
     const size_t smem = 16 * (size_t)a.nstage + sizeof(Group) * kMaxDecodePairs + 4 * (2 * kMaxDecodeT + 4) + 16 +
                         (size_t)a.T * c.H * 2 + (size_t)MT * c.I * 2 + 128 + (size_t)a.nstage * a.stage_bytes;
     auto kern = ffn_decode_kernel<FMT, MT>;
@@ -918,8 +937,8 @@ extern "C" int moe_combine(const float* y_part, int T, int k, int H, void* y_bf1
     const size_t n4 = (size_t)T * H / 4;
     const int threads = 256;
     const int blocks = (int)std::min<size_t>((n4 + threads - 1) / threads, 148 * 8);
-    combine_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(y_part, T, k, H, (uint16_t*)y_bf16);
-    MOE_CUDA_TRY(cudaGetLastError());
+    MOE_CUDA_TRY(launch_pdl(combine_kernel, dim3(blocks), dim3(threads), 0, (cudaStream_t)stream, y_part, T, k, H,
+                            (uint16_t*)y_bf16));
     return MOE_OK;
 }
 

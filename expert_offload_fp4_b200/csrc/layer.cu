@@ -1,0 +1,54 @@
+// One decode MoE layer in one host call: the per-layer sequence of the engine
+// (route, slot lookup, expert FFN, miss streaming, combine) issued natively, so
+// the host's share of a layer is a handful of driver calls.
+//
+// Order (post.smzdm.com/p/aomxznrn, "FreeToken干的事": resident experts run
+// on the GPU while missing ones cross PCIe): router and lookup are enqueued,
+// then the FFN, whose CTAs on resident experts start at once; only then does
+// the host wait (bounded) for the lookup's miss list and put the misses on the
+// copy stream; the combine follows the FFN on the compute stream.
+#include "common.cuh"
+
+using namespace moe;
+
+extern "C" int moe_decode_layer(moe_pool* p, int layer, const void* x_bf16, int T, const void* wr_bf16,
+                                const float* bias, int renormalize, int32_t* idx, float* w,
+                                int32_t* slot_of, float* y_part, void* y_bf16, int* status,
+                                void* route_ws, size_t route_ws_bytes, moe_lookup_result* res,
+                                void* copy_start, void* copy_end, int overlap, void* stream,
+                                void* copy_stream) {
+    if (!p) return fail(MOE_EINVAL, "null pool");
+    const moe_config& c = p->cfg;
+    // the caller's result arrays, else local ones of the largest size a call needs
+    int32_t uniq_l[kMaxE], hit_l[kMaxE];
+    moe_miss miss_l[kMaxE];
+    moe_lookup_result local{0, 0, uniq_l, hit_l, miss_l};
+    moe_lookup_result* r = res ? res : &local;
+    cudaStream_t cs = (cudaStream_t)copy_stream;
+    auto copies = [&]() -> int {
+        if (r->n_miss == 0) return MOE_OK;
+        if (copy_start) MOE_CUDA_TRY(cudaEventRecord((cudaEvent_t)copy_start, cs));
+        const int rc = moe_stream_misses(p, layer, r->miss_h, r->n_miss, copy_stream);
+        if (rc) return rc;
+        if (copy_end) MOE_CUDA_TRY(cudaEventRecord((cudaEvent_t)copy_end, cs));
+        return MOE_OK;
+    };
+    int rc = moe_route(x_bf16, wr_bf16, bias, T, c.H, c.E, c.k, renormalize, idx, w, route_ws,
+                       route_ws_bytes, stream);
+    if (rc) return rc;
+    if (!overlap) {
+        // misses streamed before the FFN is enqueued (for tools that serialise kernels)
+        if ((rc = moe_slot_lookup(p, layer, idx, T, c.k, slot_of, r, stream))) return rc;
+        if ((rc = copies())) return rc;
+        if ((rc = moe_expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, status, stream))) return rc;
+        return moe_combine(y_part, T, c.k, c.H, y_bf16, stream);
+    }
+    if ((rc = moe_slot_lookup_launch(p, layer, idx, T, c.k, slot_of, stream))) return rc;
+    rc = moe_expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, status, stream);
+    // the launched lookup is collected whatever the FFN launch returned
+    const int rc2 = moe_slot_lookup_result(p, r);
+    if (rc) return rc;
+    if (rc2) return rc2;
+    if ((rc = copies())) return rc;
+    return moe_combine(y_part, T, c.k, c.H, y_bf16, stream);
+}

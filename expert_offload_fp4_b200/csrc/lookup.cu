@@ -9,6 +9,7 @@
 // ascending clock order; the kernel finds them by repeated block-wide argmin.
 // Results go to slot_of (device) and to a mapped pinned host record that the
 // host waits for (bounded) to drive the copy engine.
+#include <atomic>
 #include <chrono>
 #include <thread>
 
@@ -71,8 +72,8 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(LookupArgs a) {
             a.out->n_uniq = 0;
             a.out->n_miss = 0;
             a.out->status = MOE_STATUS_BAD_EXPERT;
-            a.out->seq = a.seq;
             __threadfence_system();
+            a.out->seq = a.seq;
         }
         return;
     }
@@ -234,11 +235,12 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(LookupArgs a) {
     for (int i = tid; i < a.n; i += blockDim.x) a.slot_of[i] = uslot[umap[a.idx[i]]];
     __syncthreads();
     if (tid == 0) {
-        // the host reads the record after the kernel's completion event, which
-        // makes these mapped-memory writes visible
+        // the host polls seq in mapped memory: the record (and the miss list and
+        // slot state above) must be visible system-wide before seq is
         a.out->n_uniq = nu;
         a.out->n_miss = nm;
         a.out->status = 0;
+        __threadfence_system();
         a.out->seq = a.seq;
     }
 }
@@ -307,20 +309,30 @@ extern "C" int moe_slot_lookup_result(moe_pool* p, moe_lookup_result* res) {
     if (!p || !res) return fail(MOE_EINVAL, "null argument");
     if (!res->uniq_h || !res->is_hit_h || !res->miss_h) return fail(MOE_EINVAL, "null result arrays");
     if (!p->lk_pending) return fail(MOE_ESTATE, "no launched lookup to collect");
-    // bounded host wait: the copy engine can only be driven once the miss list is known
-    const auto t0 = std::chrono::steady_clock::now();
-    while (true) {
-        cudaError_t q = cudaEventQuery(p->lk_event);
-        if (q == cudaSuccess) break;
-        if (q != cudaErrorNotReady) {
-            p->lk_pending = 0;
-            return cuda_fail(q, "lookup kernel");
-        }
-        if (std::chrono::steady_clock::now() - t0 > std::chrono::seconds(10))
-            return fail(MOE_ETIMEOUT, "lookup kernel did not finish within 10 s");
-    }
-    p->lk_pending = 0;
+    // bounded host wait: the copy engine can only be driven once the miss list is
+    // known.  The record's seq (written last, behind a system fence) shows it as
+    // soon as the kernel writes it; the completion event catches a failed launch.
     volatile LookupOut* o = p->lk_h;
+    const auto t0 = std::chrono::steady_clock::now();
+    for (unsigned it = 0;; it++) {
+        if (o->seq == p->lk_seq) break;
+        if ((it & 63) == 63) {
+            cudaError_t q = cudaEventQuery(p->lk_event);
+            if (q == cudaSuccess) {
+                if (o->seq == p->lk_seq) break;
+                p->lk_pending = 0;
+                return fail(MOE_ECUDA, "lookup record not written");
+            }
+            if (q != cudaErrorNotReady) {
+                p->lk_pending = 0;
+                return cuda_fail(q, "lookup kernel");
+            }
+            if (std::chrono::steady_clock::now() - t0 > std::chrono::seconds(10))
+                return fail(MOE_ETIMEOUT, "lookup kernel did not finish within 10 s");
+        }
+    }
+    std::atomic_thread_fence(std::memory_order_acquire);
+    p->lk_pending = 0;
     if (o->seq != p->lk_seq) return fail(MOE_ECUDA, "lookup record not written");
     if (o->status) return fail(MOE_EBOUNDS, "expert index outside [0, E)");
     res->n_uniq = o->n_uniq;

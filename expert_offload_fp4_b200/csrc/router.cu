@@ -29,6 +29,27 @@ router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr,
     pdl_trigger();   // the slot lookup may launch now; it waits for this grid to finish
     const int t0 = blockIdx.y * TT;
     const int nt = min(TT, T - t0);
+    const int e0 = (blockIdx.x * kRouterWarps + warp) * EPW;
+
+    // H % 256 == 0, so every lane owns exactly H / 256 chunks of a row: c = lane + 32 q.
+    // They are taken kPre at a time, all loads of a batch issued before any use; the
+    // first batch (the router's own weights) before waiting for the previous kernel.
+    const int nper = H / 256;
+    constexpr int kPre = EPW == 1 ? 8 : 4;
+    uint4 pre[EPW][kPre];
+    auto load_batch = [&](int q0) {
+#pragma unroll
+        for (int a = 0; a < EPW; a++)
+#pragma unroll
+            for (int q = 0; q < kPre; q++) {
+                const int e = e0 + a;
+                pre[a][q] = (q0 + q < nper && e < E)
+                                ? __ldg(reinterpret_cast<const uint4*>(wr + size_t(e) * H) + lane + 32 * (q0 + q))
+                                : make_uint4(0, 0, 0, 0);
+            }
+    };
+    load_batch(0);
+    pdl_wait();      // x (and the buffers this kernel writes) belong to earlier kernels
 
     for (int v = threadIdx.x; v < TT * H / 8; v += blockDim.x) {
         const int t = (v * 8) / H, h = v * 8 - t * H;
@@ -43,28 +64,14 @@ router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr,
     }
     __syncthreads();
 
-    const int e0 = (blockIdx.x * kRouterWarps + warp) * EPW;
     float acc[EPW][TT];
 #pragma unroll
     for (int a = 0; a < EPW; a++)
 #pragma unroll
         for (int t = 0; t < TT; t++) acc[a][t] = 0.0f;
 
-    // H % 256 == 0, so every lane owns exactly H / 256 chunks: c = lane + 32 q.
-    // They are taken kPre at a time, all loads of a batch issued before any use.
-    const int nper = H / 256;
-    constexpr int kPre = EPW == 1 ? 8 : 4;
     for (int q0 = 0; q0 < nper; q0 += kPre) {
-        uint4 pre[EPW][kPre];
-#pragma unroll
-        for (int a = 0; a < EPW; a++)
-#pragma unroll
-            for (int q = 0; q < kPre; q++) {
-                const int e = e0 + a;
-                pre[a][q] = (q0 + q < nper && e < E)
-                                ? __ldg(reinterpret_cast<const uint4*>(wr + size_t(e) * H) + lane + 32 * (q0 + q))
-                                : make_uint4(0, 0, 0, 0);
-            }
+        if (q0 > 0) load_batch(q0);
 #pragma unroll
         for (int q = 0; q < kPre; q++) {
             if (q0 + q >= nper) break;
@@ -187,8 +194,8 @@ static cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const fl
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
     dim3 grid((E + kRouterWarps * EPW - 1) / (kRouterWarps * EPW), (T + TT - 1) / TT);
-    kern<<<grid, kRouterWarps * 32, smem, s>>>(x, wr, bias, T, H, E, k, renorm, idx, w, logits, cnt);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(kRouterWarps * 32), smem, s, x, wr, bias, T, H, E, k, renorm, idx, w,
+                      logits, cnt);
 }
 
 // Shared by the entry points that own their scratch differently.

@@ -31,9 +31,20 @@ class DecodeLayer:
         self.lookup = api.Lookup(min(T * k, E))
         self.copy_stream = torch.cuda.Stream(device=device)
         # optional timing hooks: lists that receive (start, end) CUDA events recorded
-        # around the FFN launch (compute stream) and around the miss copies (copy stream)
+        # around the miss copies (copy stream) and around the FFN launch (compute
+        # stream; setting this one issues the layer call by call from Python)
         self.ffn_events = None
         self.copy_events = None
+        self._spare_events = []
+
+    def reserve_copy_events(self, n):
+        """Create n (start, end) event pairs for the copy_events hook ahead of time
+        (torch creates a CUDA event at its first record, so each is recorded once)."""
+        for _ in range(n):
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for e in ev:
+                e.record(self.copy_stream)
+            self._spare_events.append(ev)
 
     def __call__(self, layer, x, wr, bias, stream=None):
         """x [T, H] bf16, wr [E, H] bf16, bias [E] fp32 (or None), all on the device.
@@ -45,6 +56,21 @@ class DecodeLayer:
         missed experts wait (bounded) for the slot's ready ticket that the copy
         stream writes after each expert's block lands."""
         p = self.pool
+        if self.ffn_events is None:
+            # the whole layer in one native call
+            ev = None
+            if self.copy_events is not None:
+                if not self._spare_events:
+                    self.reserve_copy_events(1)
+                ev = self._spare_events[-1]
+            api.decode_layer(p, layer, x, wr, bias, self.renormalize, self.idx, self.w, self.slot_of,
+                             self.y_part, self.y, self.status, self.ws, lookup=self.lookup,
+                             copy_events=ev, overlap=self.overlap, stream=stream,
+                             copy_stream=self.copy_stream)
+            if ev is not None and self.lookup.n_miss:
+                self.copy_events.append((self._spare_events.pop(), self.lookup.n_miss))
+            return self.y
+        # step by step, with events around the FFN launch
         api.route(x, wr, bias, p.k, self.renormalize, self.idx, self.w, self.ws, stream)
         if not self.overlap:
             api.slot_lookup(p, layer, self.idx, self.slot_of, self.lookup, stream)

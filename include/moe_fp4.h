@@ -228,13 +228,16 @@ int moe_expert_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const i
  * Process-wide; affects later launches.  Errors: MOE_EINVAL (non-positive). */
 int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
 
-/* Tracing: when buf is a device buffer of at least 8 * 148 (8 per SM) u64,
+/* Tracing: when buf is a device buffer of at least 64 * 148 (64 per SM) u64,
  * each CTA of every later moe_expert_ffn launch writes global-timer stamps (ns)
- * of its phases: [0] start, [1] the preceding kernel (the slot lookup)
+ * at row blockIdx * 64: [0] start, [1] the preceding kernel (the slot lookup)
  * complete and the activations staged, [2] expert table built,
  * [3] first item's weights landed, [4] gate/up items done and published,
- * [5] first down item's h dependency met, [6] last item done, [7] end.
- * Unwritten entries keep their old value.  NULL turns tracing off. */
+ * [5] first down item's h dependency met, [6] last item done, [7] end;
+ * for the CTA's first 16 items j: [8 + 2j] its weights landed (first consumer
+ * warp), [9 + 2j] that warp done with it, [40 + j] its copies issued; [56] the
+ * CTA's item count and [57] how many of them are gate/up items (counts, not
+ * times).  Unwritten entries keep their old value.  NULL turns tracing off. */
 int moe_set_ffn_trace(void* buf);
 
 /* Block-scaled NVFP4 GEMM on the tcgen05 tensor cores (the contraction of
@@ -280,6 +283,26 @@ int moe_prefill_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const 
  * by routing weight): y[t, :] = bf16(sum over j = 0..k-1 of y_part[t, j, :]),
  * summed in fp32 in rank order, rounded to nearest even. */
 int moe_combine(const float* y_part, int T, int k, int H, void* y_bf16, void* stream);
+
+/* One decode MoE layer in one call (the engine's per-layer sequence,
+ * post.smzdm.com/p/aomxznrn "FreeToken干的事": resident experts compute on the
+ * GPU while missing ones cross PCIe).  Runs moe_route, moe_slot_lookup_launch,
+ * moe_expert_ffn, moe_slot_lookup_result (the one host wait, bounded),
+ * moe_stream_misses on copy_stream and moe_combine, with the arguments and
+ * rules of those calls; k, H and E come from the pool.  Caller-owned device
+ * buffers: idx, w, slot_of [T, k]; y_part [T, k, H] fp32; y_bf16 [T, H];
+ * status (device int); route_ws of moe_route_workspace_bytes(T, E) bytes.
+ * res: host arrays that receive the lookup result (capacity >= min(T*k, E)),
+ * or NULL.  copy_start / copy_end: CUDA events recorded on copy_stream before
+ * and after the miss copies when the layer has misses, or NULL.  overlap = 0
+ * waits for the miss list and issues the copies before the FFN is enqueued
+ * (for tools that serialise kernels).  Returns the first failing call's error;
+ * a launched lookup is collected even when the FFN launch fails. */
+int moe_decode_layer(moe_pool* pool, int layer, const void* x_bf16, int T, const void* wr_bf16,
+                     const float* bias, int renormalize, int32_t* idx, float* w, int32_t* slot_of,
+                     float* y_part, void* y_bf16, int* status, void* route_ws,
+                     size_t route_ws_bytes, moe_lookup_result* res, void* copy_start,
+                     void* copy_end, int overlap, void* stream, void* copy_stream);
 
 /* q* split (post.smzdm.com/p/a825qpgl section 二: q* = m*B_p/B_h; "跑不快大模型，
  * 先别急着怪显卡" section 二: pull : compute = pcie_bw : (cpu_bw - pcie_bw)).

@@ -365,6 +365,50 @@ def test_decode_layer_call_with_misses_matches_oracle(m):
     pool.close()
 
 
+def test_native_layer_call_matches_step_by_step_calls(m):
+    """moe_decode_layer (one native call per layer, with and without overlap) and
+    the same layer issued call by call from Python give bit-identical outputs,
+    miss lists and LRU state; the copy-event hook records one pair per layer
+    with misses."""
+    w = small("nl", "mxfp4", H=256, I=256, E=16, k=4, L=2, zipf=0.5)
+    T = 3
+    pools, layers = [], []
+    for mode in ("native", "native_serial", "python"):
+        pool = m.Pool(w.H, w.I, w.E, w.k, w.L, w.fmt, 12, max_tokens=T)
+        for layer in range(w.L):
+            for e in range(w.E):
+                pool.load_expert(layer, e, weights(w, layer, e))
+        lo = m.DecodeLayer(pool, T, overlap=(mode != "native_serial"))
+        if mode == "python":
+            lo.ffn_events = []
+        lo.copy_events = []
+        pools.append(pool)
+        layers.append(lo)
+    for step in range(3):
+        for layer in range(w.L):
+            x = gen.activations(w, layer, step, T)
+            wr = gen.router_weight(w, layer)
+            b = gen.router_bias(w, layer)
+            outs = []
+            for lo in layers:
+                y = lo(layer, bf16(x), bf16(wr), dev(b))
+                torch.cuda.synchronize()
+                assert int(lo.status.item()) == 0
+                outs.append((host_bits(y), lo.lookup.miss_list()))
+            for o in outs[1:]:
+                assert np.array_equal(o[0], outs[0][0]) and o[1] == outs[0][1]
+    states = [p.read_state() for p in pools]
+    for st in states[1:]:
+        for key in states[0]:
+            assert np.array_equal(st[key], states[0][key]), key
+    n_layers_with_misses = len(layers[0].copy_events)
+    assert n_layers_with_misses > 0
+    assert all(len(lo.copy_events) == n_layers_with_misses for lo in layers)
+    assert all(ev[0].elapsed_time(ev[1]) >= 0.0 for ev, _ in layers[0].copy_events)
+    for p in pools:
+        p.close()
+
+
 def test_pool_reset_restricts_active_slots(m):
     """After a reset to n active slots the LRU behaves as a fresh n-slot pool."""
     E, k, L = 32, 4, 2
