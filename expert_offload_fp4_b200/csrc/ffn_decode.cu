@@ -247,11 +247,50 @@ __device__ __forceinline__ void chunk_dot_pair(const uint8_t* gcode, const uint8
     }
 }
 
+// Sum over the G lanes of each lane group (G a power of two <= 32, warp-uniform);
+// the offsets are unrolled and the MT sums interleaved.
 template <int MT>
 __device__ __forceinline__ void group_reduce(float (&acc)[MT], int G) {
 #pragma unroll
-    for (int m = 0; m < MT; m++)
-        for (int off = G >> 1; off >= 1; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+    for (int off = 16; off >= 1; off >>= 1) {
+        if (off < G) {
+#pragma unroll
+            for (int m = 0; m < MT; m++) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+        }
+    }
+}
+
+template <int MT>
+__device__ __forceinline__ void group_reduce4(float (&x0)[MT], float (&y0)[MT], float (&x1)[MT], float (&y1)[MT],
+                                              int G, bool two) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        if (off < G) {
+#pragma unroll
+            for (int m = 0; m < MT; m++) {
+                x0[m] += __shfl_xor_sync(0xffffffffu, x0[m], off);
+                y0[m] += __shfl_xor_sync(0xffffffffu, y0[m], off);
+                if (two) {
+                    x1[m] += __shfl_xor_sync(0xffffffffu, x1[m], off);
+                    y1[m] += __shfl_xor_sync(0xffffffffu, y1[m], off);
+                }
+            }
+        }
+    }
+}
+
+template <int MT>
+__device__ __forceinline__ void group_reduce2(float (&x)[MT], float (&y)[MT], int G) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        if (off < G) {
+#pragma unroll
+            for (int m = 0; m < MT; m++) {
+                x[m] += __shfl_xor_sync(0xffffffffu, x[m], off);
+                y[m] += __shfl_xor_sync(0xffffffffu, y[m], off);
+            }
+        }
+    }
 }
 
 __host__ __device__ __forceinline__ int lanes_per_row(int K) {
@@ -259,19 +298,6 @@ __host__ __device__ __forceinline__ int lanes_per_row(int K) {
     int g = 32;
     while (g > 1 && cpr % g) g >>= 1;
     return g;
-}
-
-struct StageMap {  // byte offsets of an item's tensors inside its stage
-    uint32_t codes0, scl0, codes1, scl1;     // A: gate codes/scales, up codes/scales; B: down
-    uint32_t scl0_in, scl1_in;               // start of the rows' scales inside the window
-    uint32_t bytes;
-};
-
-__device__ __forceinline__ void window(unsigned long long start, unsigned long long len,
-                                       unsigned long long& wstart, uint32_t& wlen, uint32_t& in) {
-    wstart = start & ~15ull;
-    in = (uint32_t)(start - wstart);
-    wlen = (uint32_t)(((start + len + 15) & ~15ull) - wstart);
 }
 
 __device__ __forceinline__ bool wait_ready(const FfnArgs& a, int slot, volatile unsigned int* abort_flag) {
@@ -456,52 +482,36 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
     const int b0 = (int)((long long)blockIdx.x * NB / gridDim.x);
     const int b1 = (int)((long long)(blockIdx.x + 1) * NB / gridDim.x);
     const int nmine = (a1 - a0) + (b1 - b0);
-    auto item_of = [&](int j) { return j < a1 - a0 ? a0 + j : NA + b0 + (j - (a1 - a0)); };
-
-    auto stage_map = [&](int item, unsigned long long* src, uint32_t* len, int& nsrc) -> StageMap {
-        StageMap m{};
-        const bool isB = item >= NA;
-        const int g = isB ? (item - NA) / nB_per : item / nA_per;
-        const int rb = isB ? (item - NA) % nB_per : item % nA_per;
-        const unsigned long long base = (unsigned long long)groups[g].slot * a.block_bytes;
-        if (!isB) {
-            const unsigned long long r0 = (unsigned long long)rb * a.RA;
-            unsigned long long ws;
-            uint32_t wl, in;
-            m.codes0 = 0;
-            src[0] = base + a.off[0] + r0 * codeA;
-            len[0] = (uint32_t)(a.RA * codeA);
-            window(base + a.off[1] + r0 * sclA, a.RA * sclA, ws, wl, in);
-            m.scl0 = len[0];
-            m.scl0_in = in;
-            src[1] = ws;
-            len[1] = wl;
-            m.codes1 = m.scl0 + wl;
-            src[2] = base + a.off[2] + r0 * codeA;
-            len[2] = len[0];
-            window(base + a.off[3] + r0 * sclA, a.RA * sclA, ws, wl, in);
-            m.scl1 = m.codes1 + len[2];
-            m.scl1_in = in;
-            src[3] = ws;
-            len[3] = wl;
-            m.bytes = m.scl1 + wl;
-            nsrc = 4;
-        } else {
-            const unsigned long long r0 = (unsigned long long)rb * a.RB;
-            unsigned long long ws;
-            uint32_t wl, in;
-            m.codes0 = 0;
-            src[0] = base + a.off[4] + r0 * codeB;
-            len[0] = (uint32_t)(a.RB * codeB);
-            window(base + a.off[5] + r0 * sclB, a.RB * sclB, ws, wl, in);
-            m.scl0 = len[0];
-            m.scl0_in = in;
-            src[1] = ws;
-            len[1] = wl;
-            m.bytes = m.scl0 + wl;
-            nsrc = 2;
+    // Stage layouts are the same for every item of a kind: A = gate codes, gate
+    // scales, up codes, up scales of RA rows; B = down codes, down scales of RB
+    // rows.  Every piece starts 16-byte aligned (H, I multiples of 256 and RA, RB
+    // powers of two >= 8, checked on the host), so each is one bulk copy.
+    const uint32_t lcA = (uint32_t)(a.RA * codeA), lsA = (uint32_t)(a.RA * sclA);
+    const uint32_t lcB = (uint32_t)(a.RB * codeB), lsB = (uint32_t)(a.RB * sclB);
+    const uint32_t bytesA = 2 * (lcA + lsA), bytesB = lcB + lsB;
+    // this CTA's items in order: (kind, group, row block), advanced without division
+    struct Cursor {
+        int j, isB, g, rb;
+    };
+    auto cursor_start = [&]() {
+        Cursor c{0, a1 == a0, 0, 0};
+        const int first = c.isB ? b0 : a0, per = c.isB ? nB_per : nA_per;
+        c.g = first / per;
+        c.rb = first - c.g * per;
+        return c;
+    };
+    auto cursor_next = [&](Cursor& c) {
+        c.j++;
+        if (!c.isB && c.j == a1 - a0) {
+            c.isB = 1;
+            c.g = b0 / nB_per;
+            c.rb = b0 - c.g * nB_per;
+            return;
         }
-        return m;
+        if (++c.rb == (c.isB ? nB_per : nA_per)) {
+            c.rb = 0;
+            c.g++;
+        }
     };
 
     if (warp == kNC) {
@@ -515,14 +525,13 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
             for (int g = 0; g < ng; g++)
                 if (groups[g].ready) ready_mask[g >> 5] |= 1u << (g & 31);
             fence_proxy_async_global();
-            for (int j = 0; j < nmine; j++) {
-                const int item = item_of(j);
-                const int st = j % a.nstage, round = j / a.nstage;
+            int st = 0, round = 0;
+            for (Cursor cu = cursor_start(); cu.j < nmine; cursor_next(cu)) {
+                const int j = cu.j, g = cu.g;
                 if (!mbar_wait(&empty[st], (round & 1) ^ 1, a.pipe_ns)) {
                     atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
                     *abort_flag = 1;
                 }
-                const int g = item >= NA ? (item - NA) / nB_per : item / nA_per;
                 if (!(ready_mask[g >> 5] & (1u << (g & 31)))) {
                     if (!wait_ready(a, groups[g].slot, abort_flag)) {
                         atomicOr(a.status, MOE_STATUS_READY_TIMEOUT);
@@ -531,17 +540,25 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                     ready_mask[g >> 5] |= 1u << (g & 31);
                     fence_proxy_async_global();
                 }
-                unsigned long long src[4];
-                uint32_t len[4];
-                int nsrc = 0;
-                const StageMap m = stage_map(item, src, len, nsrc);
                 uint8_t* dst = stages + (size_t)st * a.stage_bytes;
+                const uint8_t* blk = a.slots + (unsigned long long)groups[g].slot * a.block_bytes;
                 if (trace && j < 16) trace[40 + j] = globaltimer();
-                mbar_arrive_expect_tx(&full[st], m.bytes);
-                uint32_t o = 0;
-                for (int i = 0; i < nsrc; i++) {
-                    bulk_g2s(dst + o, a.slots + src[i], len[i], &full[st]);
-                    o += len[i];
+                if (!cu.isB) {
+                    const unsigned long long r0 = (unsigned long long)cu.rb * a.RA;
+                    mbar_arrive_expect_tx(&full[st], bytesA);
+                    bulk_g2s(dst, blk + a.off[0] + r0 * codeA, lcA, &full[st]);
+                    bulk_g2s(dst + lcA, blk + a.off[1] + r0 * sclA, lsA, &full[st]);
+                    bulk_g2s(dst + lcA + lsA, blk + a.off[2] + r0 * codeA, lcA, &full[st]);
+                    bulk_g2s(dst + 2 * lcA + lsA, blk + a.off[3] + r0 * sclA, lsA, &full[st]);
+                } else {
+                    const unsigned long long r0 = (unsigned long long)cu.rb * a.RB;
+                    mbar_arrive_expect_tx(&full[st], bytesB);
+                    bulk_g2s(dst, blk + a.off[4] + r0 * codeB, lcB, &full[st]);
+                    bulk_g2s(dst + lcB, blk + a.off[5] + r0 * sclB, lsB, &full[st]);
+                }
+                if (++st == a.nstage) {
+                    st = 0;
+                    round++;
                 }
             }
             // no copy may still be in flight when the CTA exits: wait (bounded) for
@@ -563,9 +580,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
             pend_n = 0;
         };
         int staged_g = -1;             // group whose h sits in hs (same on every consumer warp)
-        for (int j = 0; j < nmine; j++) {
-            const int item = item_of(j);
-            const int st = j % a.nstage, round = j / a.nstage;
+        int st = 0, round = 0;
+        for (Cursor cu = cursor_start(); cu.j < nmine; cursor_next(cu)) {
+            const int j = cu.j, g = cu.g, rb = cu.rb;
+            const bool isB = cu.isB;
             const bool ok = mbar_wait(&full[st], round & 1, a.pipe_ns);
             if (!ok) {
                 if (lane == 0) atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
@@ -573,62 +591,122 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
             }
             if (trace && tid == 0 && j == 0) trace[3] = globaltimer();
             if (trace && tid == 0 && j < 16) trace[8 + 2 * j] = globaltimer();
-            unsigned long long src[4];
-            uint32_t len[4];
-            int nsrc;
-            const StageMap m = stage_map(item, src, len, nsrc);
+            if (trace && tid == 0 && j == 1) trace[62] = clock64();
             const uint8_t* sb = stages + (size_t)st * a.stage_bytes;
-            const bool isB = item >= NA;
-            const int g = isB ? (item - NA) / nB_per : item / nA_per;
             const Group& G = groups[g];
             const int M = G.M;
             if (!isB) {
-                // A: gate row p and up row p of this item per lane group
-                if (g != pend_g) {
-                    publish();
-                    pend_g = g;
+                // A: gate row p and up row p per lane group, of this item and (when
+                // the next item is also a gate/up item) of the next one together:
+                // two independent chains per warp hide each other's latency
+                // (pairs only for up to 2 tokens per expert: more tokens already give
+                // each warp independent chains, and the registers of two would spill)
+                const int np = (MT <= 2 && j + 1 < a1 - a0) ? 2 : 1;
+                Cursor cn = cu;
+                int st2 = st, round2 = round;
+                bool ok2 = true;
+                if (np == 2) {
+                    cursor_next(cn);
+                    if (++st2 == a.nstage) {
+                        st2 = 0;
+                        round2++;
+                    }
+                    ok2 = mbar_wait(&full[st2], round2 & 1, a.pipe_ns);
+                    if (!ok2) {
+                        if (lane == 0) atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
+                        *abort_flag = 1;
+                    }
                 }
-                const int rb = item % nA_per;
+                const Group* GG[2] = {&G, &groups[cn.g]};
+                const int gg[2] = {g, cn.g}, rbs[2] = {rb, cn.rb};
+                const uint8_t* sbs[2] = {sb, stages + (size_t)st2 * a.stage_bytes};
+                const int MM[2] = {M, GG[1]->M};
                 const int RW = 32 / GA, sub = lane / GA, gl = lane % GA;
-                const __half* act[MT];
+                const __half* act[2][MT];
 #pragma unroll
-                for (int q = 0; q < MT; q++) act[q] = xs + (size_t)G.tok[q < M ? q : 0] * a.H;
+                for (int u = 0; u < 2; u++)
+#pragma unroll
+                    for (int q = 0; q < MT; q++) act[u][q] = xs + (size_t)GG[u]->tok[q < MM[u] ? q : 0] * a.H;
                 for (int base = 0; base < a.RA; base += kNC * RW) {
                     const int p = base + warp * RW + sub;
-                    float ag[MT], au[MT];
+                    float ag[2][MT], au[2][MT];
 #pragma unroll
-                    for (int q = 0; q < MT; q++) ag[q] = au[q] = 0.0f;
-                    if (p < a.RA && ok) {
-                        const uint8_t* gc = sb + m.codes0 + (size_t)p * codeA;
-                        const uint8_t* gs = sb + m.scl0 + m.scl0_in + (size_t)p * sclA;
-                        const uint8_t* uc = sb + m.codes1 + (size_t)p * codeA;
-                        const uint8_t* us = sb + m.scl1 + m.scl1_in + (size_t)p * sclA;
+                    for (int u = 0; u < 2; u++)
+#pragma unroll
+                        for (int q = 0; q < MT; q++) ag[u][q] = au[u][q] = 0.0f;
+                    if (p < a.RA && ok && ok2) {
+                        const uint8_t *gc[2], *gs[2], *uc[2], *us[2];
+#pragma unroll
+                        for (int u = 0; u < 2; u++) {
+                            gc[u] = sbs[u] + (size_t)p * codeA;
+                            gs[u] = sbs[u] + lcA + (size_t)p * sclA;
+                            uc[u] = sbs[u] + lcA + lsA + (size_t)p * codeA;
+                            us[u] = sbs[u] + 2 * lcA + lsA + (size_t)p * sclA;
+                        }
+                        if (trace && tid == 0 && j == 1) trace[58] = clock64();
+                        if (np == 2) {
+                            for (int c = gl; c < cprA; c += GA) {
+                                chunk_dot_pair<FMT, MT>(gc[0], gs[0], uc[0], us[0], c, cprA, act[0], MM[0], ag[0], au[0]);
+                                chunk_dot_pair<FMT, MT>(gc[1], gs[1], uc[1], us[1], c, cprA, act[1], MM[1], ag[1], au[1]);
+                            }
+                        } else {
 #pragma unroll 2
-                        for (int c = gl; c < cprA; c += GA)
-                            chunk_dot_pair<FMT, MT>(gc, gs, uc, us, c, cprA, act, M, ag, au);
-                    }
-                    group_reduce<MT>(ag, GA);
-                    group_reduce<MT>(au, GA);
-                    if (p < a.RA && gl == 0) {
-                        const int i = rb * a.RA + p;
-#pragma unroll
-                        for (int q = 0; q < MT; q++) {
-                            if (q >= M) break;
-                            const float xi = xinv[G.tok[q]] * 16384.0f;   // undo the decode's 2^-14
-                            const float gv = ag[q] * xi * G.ts[0];
-                            const float uv = au[q] * xi * G.ts[1];
-                            const float hv = gv / (1.0f + expf(-gv)) * uv;
-                            a.hbuf[(size_t)(G.pos + q) * a.I + i] = hv;
-                            atomicMax(a.hamax + G.pos + q, __float_as_uint(fabsf(hv)));
+                            for (int c = gl; c < cprA; c += GA)
+                                chunk_dot_pair<FMT, MT>(gc[0], gs[0], uc[0], us[0], c, cprA, act[0], MM[0], ag[0], au[0]);
                         }
                     }
-                    // rows this warp finished in this pass (the same count on every lane)
-                    const int left = a.RA - (base + warp * RW);
-                    pend_n += left <= 0 ? 0 : (left < RW ? left : RW);
+                    if (trace && tid == 0 && j == 1) trace[59] = clock64();
+                    group_reduce4<MT>(ag[0], au[0], ag[1], au[1], GA, np == 2);
+                    if (trace && tid == 0 && j == 1) trace[60] = clock64();
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        if (u >= np) break;
+                        const Group& Gu = *GG[u];
+                        if (gg[u] != pend_g) {     // rows of the previous group are all written
+                            publish();
+                            pend_g = gg[u];
+                        }
+                        if (p < a.RA && gl == 0) {
+                            const int i = rbs[u] * a.RA + p;
+#pragma unroll
+                            for (int q = 0; q < MT; q++) {
+                                if (q >= MM[u]) break;
+                                const float xi = xinv[Gu.tok[q]] * 16384.0f;   // undo the decode's 2^-14
+                                const float gv = ag[u][q] * xi * Gu.ts[0];
+                                const float uv = au[u][q] * xi * Gu.ts[1];
+                                const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+                                a.hbuf[(size_t)(Gu.pos + q) * a.I + i] = hv;
+                                atomicMax(a.hamax + Gu.pos + q, __float_as_uint(fabsf(hv)));
+                            }
+                        }
+                        // rows this warp finished in this pass (the same count on every lane)
+                        const int left = a.RA - (base + warp * RW);
+                        pend_n += left <= 0 ? 0 : (left < RW ? left : RW);
+                    }
+                    if (trace && tid == 0 && j == 1) trace[61] = clock64();
                 }
-                if (j + 1 == a1 - a0) {             // last A item of this CTA
+                if (np == 2) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[st2]);
+                }
+                if (j + np == a1 - a0) {            // last A item of this CTA
                     publish();
                     if (trace && tid == 0) trace[4] = globaltimer();
+                }
+                if (np == 2) {
+                    // release the first stage and step over both items (the loop's
+                    // increment takes the second)
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[st]);
+                    if (trace && tid == 0 && j < 16) trace[9 + 2 * j] = globaltimer();
+                    cursor_next(cu);
+                    st = st2;
+                    round = round2;
+                    if (++st == a.nstage) {
+                        st = 0;
+                        round++;
+                    }
+                    continue;
                 }
             } else {
                 // B: h of the group staged once per run of its items, then RB rows of down
@@ -663,7 +741,6 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
                     named_sync(1, kNC * 32);
                     staged_g = g;
                 }
-                const int rb = (item - NA) % nB_per;
                 const int RW = 32 / GB, sub = lane / GB, gl = lane % GB;
                 const __half* act[MT];
 #pragma unroll
@@ -674,8 +751,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
 #pragma unroll
                     for (int q = 0; q < MT; q++) ay[q] = 0.0f;
                     if (r < a.RB && ok) {
-                        const uint8_t* dc = sb + m.codes0 + (size_t)r * codeB;
-                        const uint8_t* ds = sb + m.scl0 + m.scl0_in + (size_t)r * sclB;
+                        const uint8_t* dc = sb + (size_t)r * codeB;
+                        const uint8_t* ds = sb + lcB + (size_t)r * sclB;
 #pragma unroll 2
                         for (int c = gl; c < cprB; c += GB) chunk_dot<FMT, MT>(dc, ds, c, cprB, act, M, ay);
                     }
@@ -695,6 +772,11 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArg
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
             if (trace && tid == 0 && j < 16) trace[9 + 2 * j] = globaltimer();
+            if (trace && tid == 0 && j == 1) trace[63] = clock64();
+            if (++st == a.nstage) {
+                st = 0;
+                round++;
+            }
         }
         publish();
         if (trace && tid == 0) trace[6] = globaltimer();
@@ -795,8 +877,12 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     const int minA = kNC * (32 / lanes_per_row(c.H)), minB = kNC * (32 / lanes_per_row(c.I));
     a.RA = pick_pow2_rows(std::max((int)(target / (2 * rowA)), minA), c.I, 64);
     a.RB = pick_pow2_rows(std::max((int)(target / rowB), minB), c.H, 256);
-    const size_t bytesA = 2 * ((size_t)a.RA * c.H / 2 + (((size_t)a.RA * c.H / bs + 15) / 16 + 1) * 16);
-    const size_t bytesB = (size_t)a.RB * c.I / 2 + (((size_t)a.RB * c.I / bs + 15) / 16 + 1) * 16;
+    // every piece of a stage (codes or scales of an item's rows) must be a whole
+    // number of 16-byte units so that each is one bulk copy at an aligned offset
+    if (((size_t)a.RA * c.H / bs) % 16 || ((size_t)a.RB * c.I / bs) % 16)
+        return fail(MOE_EINVAL, "decode FFN: item scale rows not a multiple of 16 bytes");
+    const size_t bytesA = 2 * ((size_t)a.RA * c.H / 2 + (size_t)a.RA * c.H / bs);
+    const size_t bytesB = (size_t)a.RB * c.I / 2 + (size_t)a.RB * c.I / bs;
     a.stage_bytes = (int)((std::max(bytesA, bytesB) + 127) / 128 * 128);
     const size_t fixed = 16 * 16 + sizeof(Group) * kMaxDecodePairs + 4 * (2 * kMaxDecodeT + 4) + 16 +
                         (size_t)a.T * c.H * 2 + (size_t)MT * c.I * 2 + 128;

@@ -237,7 +237,9 @@ int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
  * for the CTA's first 16 items j: [8 + 2j] its weights landed (first consumer
  * warp), [9 + 2j] that warp done with it, [40 + j] its copies issued; [56] the
  * CTA's item count and [57] how many of them are gate/up items (counts, not
- * times).  Unwritten entries keep their old value.  NULL turns tracing off. */
+ * times); SM clock counts (clock64) for its item 1 on the first consumer warp:
+ * [62] weights landed, [58] dot products start, [59] dot products done,
+ * [60] lane reductions done, [61] epilogue done, [63] stage released.  Unwritten entries keep their old value.  NULL turns tracing off. */
 int moe_set_ffn_trace(void* buf);
 
 /* Block-scaled NVFP4 GEMM on the tcgen05 tensor cores (the contraction of
