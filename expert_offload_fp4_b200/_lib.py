@@ -14,6 +14,7 @@ MOE_OK, MOE_EINVAL, MOE_ENOMEM, MOE_ECUDA, MOE_ETIMEOUT, MOE_EBOUNDS, MOE_ESTATE
 ERR_NAMES = {1: "MOE_EINVAL", 2: "MOE_ENOMEM", 3: "MOE_ECUDA", 4: "MOE_ETIMEOUT",
              5: "MOE_EBOUNDS", 6: "MOE_ESTATE"}
 MOE_MXFP4, MOE_NVFP4 = 0, 1
+MOE_COPY_SM, MOE_COPY_DMA = 0, 1
 STATUS_READY_TIMEOUT, STATUS_DEP_TIMEOUT, STATUS_BAD_SLOT, STATUS_BAD_EXPERT, STATUS_PIPE_TIMEOUT = 1, 2, 4, 8, 16
 
 
@@ -68,6 +69,7 @@ SIGNATURES = {
     "moe_slot_lookup_launch": (i32, [vp, i32, vp, i32, i32, vp, vp]),
     "moe_slot_lookup_result": (i32, [vp, C.POINTER(LookupResult)]),
     "moe_stream_misses": (i32, [vp, i32, C.POINTER(Miss), i32, vp]),
+    "moe_pool_set_copy_mode": (i32, [vp, i32]),
     "moe_expert_ffn": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp]),
     "moe_combine": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_decode_layer": (i32, [vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,

@@ -77,6 +77,11 @@ class Pool:
         L.check("moe_pool_reset", self.lib.moe_pool_reset(self.handle, n))
         self.n_active = n
 
+    def set_copy_mode(self, mode):
+        """"sm" (a kernel reads the mapped host block over PCIe) or "dma" (copy engine)."""
+        m = {"sm": L.MOE_COPY_SM, "dma": L.MOE_COPY_DMA}[mode]
+        L.check("moe_pool_set_copy_mode", self.lib.moe_pool_set_copy_mode(self.handle, m))
+
     def read_state(self):
         sk = np.empty(self.n_slots, np.int32)
         sc = np.empty(self.n_slots, np.uint64)

@@ -60,6 +60,8 @@ int preload_lookup_kernels();
 int preload_ffn_kernels();
 int preload_gemm_kernels();
 int preload_prefill_kernels();
+int preload_pull_kernels();
+cudaError_t launch_pull(const uint8_t* src_d, uint8_t* dst, size_t bytes, int num_sms, cudaStream_t s);
 
 }  // namespace moe
 
@@ -71,10 +73,13 @@ struct moe_pool {
     int n_active;                 // slots the LRU may use (<= cfg.n_slots)
     int device;
     int num_sms;
+    int ffn_smem;                 // shared-memory bytes the decode FFN may take per CTA
     // storage
     uint8_t* slots;               // device [n_slots][block]
-    uint8_t* host;                // pinned [host_layers][E][block]
+    uint8_t* host;                // pinned, mapped [host_layers][E][block]
+    const uint8_t* host_d;        // its device alias (read by the pull kernel)
     uint8_t* host_loaded;         // host flags [host_layers * E]
+    int copy_mode;                // MOE_COPY_SM or MOE_COPY_DMA
     // LRU metadata (device)
     int32_t* slot_key;            // [n_slots]
     unsigned long long* slot_clock;  // [n_slots]

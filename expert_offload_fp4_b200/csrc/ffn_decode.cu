@@ -27,6 +27,10 @@ namespace moe {
 
 constexpr int kNC = 8;                       // consumer warps
 constexpr int kFfnThreads = (kNC + 1) * 32;  // + one producer warp
+// Register cap: with 9 warps one SM sub-partition holds 3 of them, and it must
+// keep room (2 x 32 x 32 registers) for warps of the miss-copy kernel the FFN
+// waits for: 3 * 32 * 144 + 2048 <= 16384.
+constexpr int kFfnMaxRegs = 144;
 constexpr int kAbortIdx = kMaxDecodePairs;   // ctr[kAbortIdx] = abort flag
 constexpr int kDoneIdx = kMaxDecodePairs + 1;
 
@@ -313,7 +317,7 @@ __device__ __forceinline__ bool wait_ready(const FfnArgs& a, int slot, volatile 
 }
 
 template <int FMT, int MT>
-__global__ void __launch_bounds__(kFfnThreads, 1) ffn_decode_kernel(const FfnArgs a) {
+__global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + a.nstage;
@@ -886,7 +890,7 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     a.stage_bytes = (int)((std::max(bytesA, bytesB) + 127) / 128 * 128);
     const size_t fixed = 16 * 16 + sizeof(Group) * kMaxDecodePairs + 4 * (2 * kMaxDecodeT + 4) + 16 +
                         (size_t)a.T * c.H * 2 + (size_t)MT * c.I * 2 + 128;
-    const size_t budget = 227 * 1024;
+    const size_t budget = (size_t)p->ffn_smem;
     if (fixed + 2 * (size_t)a.stage_bytes > budget) return fail(MOE_EINVAL, "decode FFN: shapes exceed shared memory");
     a.nstage = (int)std::min<size_t>(12, (budget - fixed) / a.stage_bytes);
     // the prologue keeps its per-(token, rank) table (7 ints + 3 floats each) in the ring
@@ -900,6 +904,8 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
         // once per pool and template: the largest shared-memory carve-out, and the
         // number of co-resident CTAs per SM at that size (1: the kernel is persistent)
         MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget));
+        MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          cudaSharedmemCarveoutMaxShared));
         int per_sm = 0;
         MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFfnThreads, budget));
         p->ffn_per_sm[fi][mi] = per_sm;
@@ -909,26 +915,14 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     if (per_sm < 1) return fail(MOE_EINVAL, "decode FFN kernel does not fit on an SM");
     const int items_max = a.T * a.k * (c.I / a.RA + c.H / a.RB);
     const int grid = std::max(1, std::min(p->num_sms * per_sm, items_max));
-    static int pdl_ok = 1;   // cleared if the driver rejects cooperative + programmatic launch
-    if (pdl_ok) {
-        cudaLaunchConfig_t lc = {};
-        lc.gridDim = dim3(grid);
-        lc.blockDim = dim3(kFfnThreads);
-        lc.dynamicSmemBytes = smem;
-        lc.stream = s;
-        cudaLaunchAttribute at[2];
-        at[0].id = cudaLaunchAttributeCooperative;
-        at[0].val.cooperative = 1;
-        at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        at[1].val.programmaticStreamSerializationAllowed = 1;
-        lc.attrs = at;
-        lc.numAttrs = 2;
-        if (cudaLaunchKernelEx(&lc, kern, a) == cudaSuccess) return MOE_OK;
-        cudaGetLastError();
-        pdl_ok = 0;
-    }
-    void* args[] = {(void*)&a};
-    MOE_CUDA_TRY(cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kFfnThreads), args, smem, s));
+    // CTAs wait on one another (down rows wait for every gate/up row of their
+    // expert), so all of them must be resident together: one CTA per SM fits
+    // (the shared-memory ring takes the SM) and the grid is at most the SM
+    // count, so they are, once the kernels ahead of this one in the stream have
+    // left.  A plain launch (not a cooperative one) lets the slot lookup before
+    // it hand over through programmatic serialisation and lets the miss copies
+    // of the copy stream run beside it; every wait is bounded in any case.
+    MOE_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(kFfnThreads), smem, s, a));
     return MOE_OK;
 }
 

@@ -110,6 +110,16 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
     p->n_active = cfg->n_slots;
     cudaGetDevice(&p->device);
     cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device);
+    {
+        // the decode FFN (one CTA per SM) leaves room for the shared-memory
+        // reservation of one more CTA, so that the miss-copy kernel it waits for
+        // can run beside it on every SM
+        int per_sm = 0, reserved = 0, optin = 0;
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, p->device);
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, p->device);
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, p->device);
+        p->ffn_smem = std::min(optin, per_sm - 2 * reserved - 1024);
+    }
     const size_t S = cfg->n_slots, LE = size_t(cfg->L) * cfg->E;
     const size_t host_bytes = size_t(p->host_layers) * cfg->E * p->lay.bytes;
     cudaError_t e;
@@ -139,13 +149,20 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
     cudaMemset(p->tscale, 0, LE * 3 * sizeof(float));
     cudaMemset(p->hamax, 0, kMaxDecodePairs * sizeof(unsigned int));
     cudaMemset(p->ctr, 0, (kMaxDecodePairs + 8) * sizeof(unsigned int));
-    e = cudaHostAlloc((void**)&p->host, host_bytes, cudaHostAllocDefault);
+    e = cudaHostAlloc((void**)&p->host, host_bytes, cudaHostAllocMapped);
     if (e != cudaSuccess) {
         p->host = nullptr;
         rc = cuda_fail(e, "cudaHostAlloc (pinned expert store)");
         moe_pool_destroy(p);
         return rc;
     }
+    {
+        void* hd = nullptr;
+        e = cudaHostGetDevicePointer(&hd, p->host, 0);
+        if (e != cudaSuccess) { rc = cuda_fail(e, "cudaHostGetDevicePointer (expert store)"); moe_pool_destroy(p); return rc; }
+        p->host_d = (const uint8_t*)hd;
+    }
+    p->copy_mode = MOE_COPY_DMA;
     e = cudaHostAlloc((void**)&p->lk_h, sizeof(LookupOut), cudaHostAllocMapped);
     if (e != cudaSuccess) {
         p->lk_h = nullptr;
@@ -167,7 +184,7 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
         return rc;
     }
     if ((rc = preload_router_kernels()) || (rc = preload_lookup_kernels()) || (rc = preload_ffn_kernels()) ||
-        (rc = preload_gemm_kernels()) || (rc = preload_prefill_kernels())) {
+        (rc = preload_gemm_kernels()) || (rc = preload_prefill_kernels()) || (rc = preload_pull_kernels())) {
         moe_pool_destroy(p);
         return rc;
     }
@@ -274,12 +291,23 @@ extern "C" int moe_stream_misses(moe_pool* p, int layer, const moe_miss* miss_h,
         const moe_miss& m = miss_h[i];
         const uint8_t* src = p->host + (size_t(hl) * c.E + m.expert) * p->lay.bytes;
         uint8_t* dst = p->slots + size_t(m.slot) * p->lay.bytes;
-        MOE_CUDA_TRY(cudaMemcpyAsync(dst, src, p->lay.bytes, cudaMemcpyHostToDevice, s));
+        if (p->copy_mode == MOE_COPY_DMA) {
+            MOE_CUDA_TRY(cudaMemcpyAsync(dst, src, p->lay.bytes, cudaMemcpyHostToDevice, s));
+        } else {
+            MOE_CUDA_TRY(launch_pull(p->host_d + (src - p->host), dst, p->lay.bytes, p->num_sms, s));
+        }
         CUresult r = wv((CUstream)s, (CUdeviceptr)(p->ready + m.slot), m.ticket, 0);
         if (r != CUDA_SUCCESS) return fail(MOE_ECUDA, "cuStreamWriteValue32 failed");
         p->stats.h2d_bytes += (long long)p->lay.bytes;
         p->stats.h2d_copies += 1;
     }
+    return MOE_OK;
+}
+
+extern "C" int moe_pool_set_copy_mode(moe_pool* p, int mode) {
+    if (!p) return fail(MOE_EINVAL, "null pool");
+    if (mode != MOE_COPY_SM && mode != MOE_COPY_DMA) return fail(MOE_EINVAL, "copy mode: MOE_COPY_SM or MOE_COPY_DMA");
+    p->copy_mode = mode;
     return MOE_OK;
 }
 

@@ -53,6 +53,13 @@ enum {
  * description (E2M1 codes, E4M3 scale per 16, FP32 tensor scale). */
 enum { MOE_MXFP4 = 0, MOE_NVFP4 = 1 };
 
+/* How moe_stream_misses moves a missed expert's block host -> slot. */
+enum {
+    MOE_COPY_SM = 0,   /* a kernel on the copy stream reads the mapped host block over
+                          PCIe with 16-byte loads from every SM */
+    MOE_COPY_DMA = 1   /* one cudaMemcpyAsync per miss on the copy engine (default) */
+};
+
 /* Bits of the device status word written by moe_expert_ffn. */
 enum {
     MOE_STATUS_READY_TIMEOUT = 1,  /* a missed expert's ready flag never arrived */
@@ -209,6 +216,13 @@ int moe_slot_lookup_result(moe_pool* pool, moe_lookup_result* res);
  * loads all of the library's kernels when it is created.  Errors: MOE_EBOUNDS, MOE_ESTATE (expert never loaded). */
 int moe_stream_misses(moe_pool* pool, int layer, const moe_miss* miss_h, int n_miss,
                       void* copy_stream);
+
+/* Select how moe_stream_misses copies (MOE_COPY_SM or MOE_COPY_DMA) for later
+ * calls on this pool.  Both write the same bytes and publish the same ready
+ * tickets.  The copy kernel of MOE_COPY_SM runs beside a waiting decode FFN
+ * (one 128-thread CTA per SM fits next to an FFN CTA: the FFN caps its
+ * registers and shared memory for that).  Errors: MOE_EINVAL. */
+int moe_pool_set_copy_mode(moe_pool* pool, int mode);
 
 /* Decode expert FFN (post.smzdm.com/p/aomxznrn: decode is bandwidth-bound and
  * scheduled apart from prefill).  For every (t, j): y_part[t, j, :] =

@@ -409,6 +409,38 @@ def test_native_layer_call_matches_step_by_step_calls(m):
         p.close()
 
 
+@pytest.mark.parametrize("mode", ["sm", "dma"])
+def test_copy_modes_fill_slots_identically(m, mode):
+    """Both miss-copy paths (SM loads of the mapped host store, copy engine) put
+    the expert's exact host bytes into the slot and give oracle-exact outputs."""
+    w = small("cm", "nvfp4", H=512, I=256, E=16, k=4, L=2, zipf=0.3)
+    T = 2
+    pool = m.Pool(w.H, w.I, w.E, w.k, w.L, w.fmt, 8, max_tokens=T)
+    pool.set_copy_mode(mode)
+    for layer in range(w.L):
+        for e in range(w.E):
+            pool.load_expert(layer, e, weights(w, layer, e))
+    lo = m.DecodeLayer(pool, T)
+    for step in range(2):
+        for layer in range(w.L):
+            x = gen.activations(w, layer, step, T)
+            wr = gen.router_weight(w, layer)
+            b = gen.router_bias(w, layer)
+            lo(layer, bf16(x), bf16(wr), dev(b))
+            torch.cuda.synchronize()
+            check_layer(w, lo, x, wr, b, layer)
+            for e, slot, _, _ in lo.lookup.miss_list():
+                for which, name in enumerate(("gate", "up", "down")):
+                    codes, scales, ts = weights(w, layer, e)[name]
+                    rows, K = codes.shape[0], codes.shape[1] * 2
+                    out = torch.empty((rows, K), dtype=torch.float32, device="cuda")
+                    m.dequant_slot(pool, slot, layer * w.E + e, which, out)
+                    ref = oracle.dequant(w.fmt, codes, scales, ts)
+                    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+    assert pool.stats()["misses"] > 0
+    pool.close()
+
+
 def test_pool_reset_restricts_active_slots(m):
     """After a reset to n active slots the LRU behaves as a fresh n-slot pool."""
     E, k, L = 32, 4, 2
