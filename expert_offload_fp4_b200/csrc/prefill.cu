@@ -236,15 +236,18 @@ struct PSmem {
     static constexpr int total = tmem_slot + 16;
 };
 
+// 128 rows x 16 scale bytes (row m: the 4 scales of each of the stage's four K=64
+// blocks) -> four 512-byte scale-factor atoms (atom s, 16-byte row r: the block-s
+// scales of rows r, r+32, r+64, r+96).  One warp; 16-byte loads and stores, no
+// bank conflicts.
 __device__ __forceinline__ void p_arrange_sf(const uint8_t* canon, uint8_t* atom, int lane) {
+    uint4 v[4];
 #pragma unroll
-    for (int q = 0; q < 4; q++) {
-        const int m = lane + 32 * q;
-        const uint4 v = *reinterpret_cast<const uint4*>(canon + 16 * m);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int s = 0; s < 4; s++) *reinterpret_cast<uint32_t*>(atom + 512 * s + 16 * lane + 4 * q) = w[s];
-    }
+    for (int q = 0; q < 4; q++) v[q] = *reinterpret_cast<const uint4*>(canon + 16 * (lane + 32 * q));
+    *reinterpret_cast<uint4*>(atom + 16 * lane) = make_uint4(v[0].x, v[1].x, v[2].x, v[3].x);
+    *reinterpret_cast<uint4*>(atom + 512 + 16 * lane) = make_uint4(v[0].y, v[1].y, v[2].y, v[3].y);
+    *reinterpret_cast<uint4*>(atom + 1024 + 16 * lane) = make_uint4(v[0].z, v[1].z, v[2].z, v[3].z);
+    *reinterpret_cast<uint4*>(atom + 1536 + 16 * lane) = make_uint4(v[0].w, v[1].w, v[2].w, v[3].w);
 }
 
 struct GemmArgs {
@@ -262,8 +265,8 @@ struct GemmArgs {
 
 // Persistent, warp-specialised grouped GEMM over the (M tile, N tile) list of
 // this call; CTA c takes tiles c, c + grid, ...  Warp 0 streams every tile's K
-// steps through the stage ring without pausing between tiles; warp 2 turns the
-// scale rows into scale-factor atoms; warp 1 issues the MMAs into one of two
+// steps through the stage ring without pausing between tiles; warps 2 and 3 turn
+// the A and B scale rows into scale-factor atoms; warp 1 issues the MMAs into one of two
 // TMEM accumulators, so warps 4-7 drain tile i while tile i+1 is multiplied.
 // MODE 1: gate/up with the SiLU * up + NVFP4 epilogue; MODE 2: down with the
 // routing-weight reduction into y.
@@ -287,7 +290,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&sfready[s], 1);
+            mbar_init(&sfready[s], 2);
             mbar_init(&empty[s], 1);
         }
         mbar_init(&accf[0], 1);
@@ -332,17 +335,32 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
                 }
             }
         }
-    } else if (warp == 2) {
+    } else if (warp == 2 || warp == 3) {
+        // warp 2 arranges the A scales, warp 3 the B scales of every stage, and
+        // copies them into the stage's TMEM scale columns itself; the commit
+        // arrives on sfready once the copies are done, so the MMA warp issues
+        // only the MMAs
+        const int off_sf = warp == 2 ? PSmem::a_sf : PSmem::b_sf;
+        const int off_atom = warp == 2 ? PSmem::a_atom : PSmem::b_atom;
+        const uint32_t col = warp == 2 ? 0u : 16u;
         int it = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             for (int kt = 0; kt < KT; kt++, it++) {
                 const int s = it % kPStages, r = it / kPStages;
                 if (!mbar_wait(&full[s], r & 1, g.limit_ns) && lane == 0) atomicOr(g.status, 1 << 16);
-                p_arrange_sf(sm + PSmem::a_sf + s * 2048, sm + PSmem::a_atom + s * 2048, lane);
-                p_arrange_sf(sm + PSmem::b_sf + s * 2048, sm + PSmem::b_atom + s * 2048, lane);
+                p_arrange_sf(sm + off_sf + s * 2048, sm + off_atom + s * 2048, lane);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sfready[s]);
+                if (lane == 0) {
+                    // the stage's previous MMAs (which read these columns) completed
+                    // before its loads were reissued, which the full wait above saw
+                    tc_fence_after();
+                    const uint32_t sf = tbase + 256 + s * 32 + col;
+#pragma unroll
+                    for (int i = 0; i < 4; i++)
+                        tmem_cp_sf_atom(sf + 4 * i, smem_desc(sm + off_atom + s * 2048 + 512 * i, 16, 128, 0));
+                    tc_commit(&sfready[s]);
+                }
             }
         }
     } else if (warp == 1) {
@@ -359,11 +377,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
                     if (!mbar_wait(&sfready[s], r & 1, g.limit_ns)) atomicOr(g.status, 1 << 16);
                     tc_fence_after();
                     const uint32_t sfa = tbase + 256 + s * 32, sfb = sfa + 16;
-#pragma unroll
-                    for (int i = 0; i < 4; i++) {
-                        tmem_cp_sf_atom(sfa + 4 * i, smem_desc(sm + PSmem::a_atom + s * 2048 + 512 * i, 16, 128, 0));
-                        tmem_cp_sf_atom(sfb + 4 * i, smem_desc(sm + PSmem::b_atom + s * 2048 + 512 * i, 16, 128, 0));
-                    }
                     const uint64_t ad = smem_desc(sm + PSmem::a_codes + s * 16384, 16, 1024, 2);
                     const uint64_t bd = smem_desc(sm + PSmem::b_codes + s * 16384, 16, 1024, 2);
 #pragma unroll
