@@ -457,6 +457,14 @@ def offload_mode(args):
 
 # ---------------------------------------------------------------------- main
 
+def decode_config(w, T, world):
+    """The `config` object of the decode line (both arms)."""
+    return {"workload": w.name, "layers": w.L, "batch": T, "format": w.fmt,
+            "slot_pool": f"{W.n_slots(w)} slots (25% of {w.L * w.E})",
+            "zipf_s": w.zipf_s, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2: ~1 GB of expert weights per step"}
+
+
 def profiled_traffic_ratio(profile, source):
     """DRAM bytes per algorithmic byte from a committed ncu summary, or None.
 
@@ -521,7 +529,7 @@ def main():
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 1000.0 * T / cb["value"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": w.name, "layers": w.L, "batch": T, "format": w.fmt},
+                "config": decode_config(w, T, args.gpus),
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0},
@@ -631,12 +639,9 @@ def main():
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16/f32",
             "data": "synthetic",
-            "config": {"workload": w.name, "layers": w.L, "batch": T, "format": w.fmt,
-                       "slot_pool": f"{W.n_slots(w)} slots (25% of {w.L * w.E})",
-                       "zipf_s": w.zipf_s, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2: ~1 GB of expert weights per step"},
+            "config": decode_config(w, T, world),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                          "kernel": "ffn_decode_kernel", "peak_source": peak_kind,

@@ -119,14 +119,25 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const int32_t* __res
         ws.cursor[e] = 0;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int e = idx[i];
-        if (e < 0 || e >= E) {
-            atomicOr(status, MOE_STATUS_BAD_EXPERT);
-            continue;
+    // eight entries per thread per round, their loads issued before any is used
+    for (int i0 = threadIdx.x; i0 < n; i0 += 8 * blockDim.x) {
+        int ev[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = i0 + u * blockDim.x;
+            ev[u] = i < n ? idx[i] : -2;
         }
-        atomicAdd(&s_cnt[e], 1);
-        ws.slot_e[e] = slot_of[i];   // every entry of an expert names the same slot
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int e = ev[u];
+            if (e == -2) continue;
+            if (e < 0 || e >= E) {
+                atomicOr(status, MOE_STATUS_BAD_EXPERT);
+                continue;
+            }
+            // every entry of an expert names the same slot: the first one records it
+            if (atomicAdd(&s_cnt[e], 1) == 0) ws.slot_e[e] = slot_of[i0 + u * blockDim.x];
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -150,6 +161,12 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const int32_t* __res
             ws.tile_row0[s_tiles[e] + t] = ws.row_off[e] + 128 * t;
         }
     }
+    __syncthreads();
+    // rows of an expert's last tile past its count are padding (no token)
+    for (int i = threadIdx.x; i < E * 128; i += blockDim.x) {
+        const int e = i >> 7, r = i & 127, c = s_cnt[e];
+        if (r < (c + 127) / 128 * 128 - c) ws.perm_tok[128 * s_tiles[e] + c + r] = -1;
+    }
 }
 
 // ---------------------------------------------------------------- quantise + scatter
@@ -158,38 +175,48 @@ __global__ void __launch_bounds__(256) prefill_quant_kernel(const uint16_t* __re
                                                            int E, const int32_t* __restrict__ idx, PrefillWs ws,
                                                            uint8_t* __restrict__ out_codes,
                                                            uint8_t* __restrict__ out_scales,
-                                                           float* __restrict__ out_sx) {
+                                                           float* __restrict__ out_sx, float* __restrict__ y0) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (warp >= T) return;
     const int t = warp;
     const uint16_t* xr = x + (size_t)t * H;
     float amax = 0.0f;
-    for (int h = lane * 8; h < H; h += 256) {
-        const uint4 q = *reinterpret_cast<const uint4*>(xr + h);
-        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+    // H / 256 (<= 16 for H <= 4096) 16-byte loads per lane, four issued at a time
+    for (int h0 = lane * 8; h0 < H; h0 += 4 * 256) {
+        uint4 q[4];
 #pragma unroll
-        for (int i = 0; i < 4; i++)
-            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(u[i] << 16)), fabsf(__uint_as_float(u[i] & 0xFFFF0000u))));
+        for (int u = 0; u < 4; u++) q[u] = h0 + u * 256 < H ? *reinterpret_cast<const uint4*>(xr + h0 + u * 256)
+                                                            : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const uint32_t w4[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[i] << 16)), fabsf(__uint_as_float(w4[i] & 0xFFFF0000u))));
+        }
+    }
+    if (y0) {   // the down GEMM accumulates into y: zero this token's row here
+        float4* yr = reinterpret_cast<float4*>(y0 + (size_t)t * H);
+        for (int v = lane; v < H / 4; v += 32) yr[v] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const float S = amax / 2688.0f;
     int rows[kMaxK];
     if (idx) {
-        for (int j = 0; j < k; j++) {
-            int r = -1;
-            if (lane == 0) {
-                const int e = idx[t * k + j];
-                if (e >= 0 && e < E) {          // invalid ids are reported by the planner
-                    const int pos = atomicAdd(ws.cursor + e, 1);
-                    r = ws.row_off[e] + pos;
-                    ws.perm_tok[r] = t;
-                    ws.perm_rank[r] = j;
-                    ws.perm_sx[r] = S;
-                }
+        // lane j claims the row of rank j (the k claims run in parallel)
+        int r = -1;
+        if (lane < k) {
+            const int e = idx[t * k + lane];
+            if (e >= 0 && e < E) {              // invalid ids are reported by the planner
+                const int pos = atomicAdd(ws.cursor + e, 1);
+                r = ws.row_off[e] + pos;
+                ws.perm_tok[r] = t;
+                ws.perm_rank[r] = lane;
+                ws.perm_sx[r] = S;
             }
-            rows[j] = __shfl_sync(0xffffffffu, r, 0);
         }
+        for (int j = 0; j < k; j++) rows[j] = __shfl_sync(0xffffffffu, r, j);
     }
     // 16-element blocks, lane-strided
     for (int b = lane; b < H / 16; b += 32) {
@@ -518,7 +545,7 @@ extern "C" int moe_nvfp4_quantize(const void* x_bf16, int T, int H, uint8_t* cod
     PrefillWs ws{};
     const int blocks = (T * 32 + 255) / 256;
     prefill_quant_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>((const uint16_t*)x_bf16, T, H, 0, 0, nullptr, ws,
-                                                                   codes, scales, sx);
+                                                                   codes, scales, sx, nullptr);
     MOE_CUDA_TRY(cudaGetLastError());
     return MOE_OK;
 }
@@ -559,12 +586,10 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
     ws.hsf = base + PL.off[13];
     ws.R = PL.R;
     ws.MT = PL.MT;
-    MOE_CUDA_TRY(cudaMemsetAsync(ws.perm_tok, 0xFF, size_t(PL.R) * 4, s));
-    MOE_CUDA_TRY(cudaMemsetAsync(y, 0, size_t(T) * c.H * sizeof(float), s));
     prefill_plan_kernel<<<1, 1024, 0, s>>>(idx, slot_of, T * c.k, c.E, ws, status);
     MOE_CUDA_TRY(cudaGetLastError());
     prefill_quant_kernel<<<(T * 32 + 255) / 256, 256, 0, s>>>((const uint16_t*)x_bf16, T, c.H, c.k, c.E, idx, ws,
-                                                              nullptr, nullptr, nullptr);
+                                                              nullptr, nullptr, nullptr, y);
     MOE_CUDA_TRY(cudaGetLastError());
 
     const size_t pool_bytes = size_t(c.n_slots) * B.bytes;
