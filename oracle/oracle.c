@@ -42,9 +42,13 @@
  *    amax(x_t)/(6*448); h quantised to NVFP4 with tensor scale 1.0;
  *  - q*: q_gpu = min(m, floor(m*B_p/B_h + 0.5)), q_cpu = m - q_gpu.
  *
- * Parity status: the codecs, router, top-k, LRU, q* and the sparse/dense MoE
- * identity are pinned by tests; the FFN numerics beyond the dense brute-force
- * identity are "parity unpinned" (the pages print no worked example).
+ * Parity status: every function is pinned by tests against what the pages and the
+ * mathematics fix: the codecs by the OCP tables and exhaustive byte sweeps, q* by
+ * the pages' printed table, the router by an fp32 error bound around the exact dot
+ * product and a full sort, the LRU by a textbook list LRU on random traces, the
+ * expert FFN by closed forms on structured experts and by the sparse = dense
+ * brute-force identity, the prefill path by closed forms on inputs NVFP4 holds
+ * exactly.  The pages print no worked example of the FFN itself.
  */
 #include <math.h>
 #include <stdint.h>
