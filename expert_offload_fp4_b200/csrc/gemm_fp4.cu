@@ -221,10 +221,13 @@ extern "C" int moe_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, c
     if ((rc = make_tmap_2d(&msa, a_scales, K / 16, M, K / 16, 16, 128, false))) return rc;
     if ((rc = make_tmap_2d(&msb, b_scales, K / 16, N, K / 16, 16, 128, false))) return rc;
     const int smem = GemmSmem::total + 1024;
-    static bool attr = false;
-    if (!attr) {
+    // the shared-memory limit is a per-device setting: raise it once per device
+    static bool attr_done[64] = {};
+    int dev = 0;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
         MOE_CUDA_TRY(cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-        attr = true;
+        if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
     dim3 grid(N / kBN, M / kBM);
     nvfp4_gemm_kernel<<<grid, kGemmThreads, smem, (cudaStream_t)stream>>>(ma, mb, msa, msb, M, N, K, D, status,

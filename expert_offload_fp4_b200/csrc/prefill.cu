@@ -525,6 +525,10 @@ int preload_prefill_kernels() {
     MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, prefill_quant_kernel));
     MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, grouped_gemm_kernel<1>));
     MOE_CUDA_TRY(cudaFuncGetAttributes(&fa, grouped_gemm_kernel<2>));
+    // on the pool's device (current while the pool is created)
+    const int smem = PSmem::total + 1024;
+    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     return MOE_OK;
 }
 
@@ -622,13 +626,7 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
     g.b_up_row = B.off[2] / gr;
     g.b_gsf_row = B.off[1] / gs;
     g.b_usf_row = B.off[3] / gs;
-    const int smem = PSmem::total + 1024;
-    static bool attr = false;
-    if (!attr) {
-        MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-        MOE_CUDA_TRY(cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-        attr = true;
-    }
+    const int smem = PSmem::total + 1024;   // the limit was raised when the pool was created
     g.NT = c.I / 64;
     const int grid1 = std::min(PL.MT * g.NT, p->num_sms);
     grouped_gemm_kernel<1><<<grid1, kPThreads, smem, s>>>(ma1, msa1, mb1, msb1, g);

@@ -91,4 +91,8 @@ def test_route_argument_checks_need_no_gpu(lib):
     assert L.moe_route(odd, p, None, 4, 256, 16, 2, 1, p, p, p, ws, None) == lib.MOE_EINVAL
     assert b"aligned" in L.moe_last_error()
     assert L.moe_combine(p, 4, 2, 254, p, None) == lib.MOE_EINVAL
+    # the per-layer call and the copy-mode setter need a pool
+    assert L.moe_decode_layer(None, 0, p, 1, p, None, 1, p, p, p, p, p, p, p, 64, None, None, None, 1,
+                              None, None) == lib.MOE_EINVAL
+    assert L.moe_pool_set_copy_mode(None, lib.MOE_COPY_DMA) == lib.MOE_EINVAL
     assert L.moe_set_wait_limits(-1.0, 1.0, 1.0) == lib.MOE_EINVAL
