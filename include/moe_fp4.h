@@ -228,10 +228,18 @@ int moe_pool_set_copy_mode(moe_pool* pool, int mode);
  * scheduled apart from prefill).  For every (t, j): y_part[t, j, :] =
  * w[t,j] * Wd (silu(Wg x_t) * (Wu x_t)) of expert idx[t,j] read from slot
  * slot_of[t,j]; FP4 weights dequantised on the fly (MXFP4: e2m1 * 2^(s-127);
- * NVFP4: e2m1 * e4m3(s) * S_tensor), fp32 accumulation.  One persistent kernel
- * with a TMA-bulk / shared-memory pipeline; waits are bounded and failures set
- * bits of *status (device int, caller-zeroed; MOE_STATUS_*).  y_part is
- * [T, k, H] fp32.  Limits: T <= max_tokens of the pool.  Errors: MOE_EINVAL. */
+ * NVFP4: e2m1 * e4m3(s) * S_tensor): exact f16 products summed in f16 within a
+ * scale block, block sums scaled and accumulated in fp32, h rounded to f16 with a
+ * per-token power-of-two scale.  One persistent kernel, one CTA per SM, fed by
+ * bulk copies into a shared-memory ring; its CTAs wait on one another (down rows
+ * need all gate/up rows of their expert) and on the ready tickets of missed
+ * experts.  It is a plain launch with programmatic stream serialisation: it
+ * stages x while the kernel before it (the slot lookup) finishes.  Waits are
+ * bounded (moe_set_wait_limits) and failures set bits of *status (device int,
+ * caller-zeroed; MOE_STATUS_*): if other work keeps one of its CTAs off the GPU
+ * for longer than the limits, the call reports a timeout instead of hanging.
+ * y_part is [T, k, H] fp32.  Limits: T <= max_tokens of the pool.
+ * Errors: MOE_EINVAL. */
 int moe_expert_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const int32_t* idx,
                    const float* w, const int32_t* slot_of, float* y_part, int* status,
                    void* stream);
