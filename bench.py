@@ -456,6 +456,47 @@ def offload_mode(args):
 
 # ---------------------------------------------------------------------- main
 
+def host_bandwidth_gbs(nbytes=1 << 30, reps=3):
+    """Host-memory bandwidth (GB/s of bytes read) of a copy split over the host's
+    cores; the best of `reps`."""
+    from concurrent.futures import ThreadPoolExecutor
+    n = max(1, min(32, os.cpu_count() or 1))
+    src = np.ones(nbytes, np.uint8)
+    dst = np.empty_like(src)
+    parts = np.array_split(np.arange(nbytes), n)
+    bounds = [(int(q[0]), int(q[-1]) + 1) for q in parts if len(q)]
+
+    def cp(b):
+        np.copyto(dst[b[0]:b[1]], src[b[0]:b[1]])
+
+    best = 0.0
+    with ThreadPoolExecutor(n) as ex:
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            list(ex.map(cp, bounds))
+            best = max(best, nbytes / (time.perf_counter() - t0) / 1e9)
+    return best, n
+
+
+def qstar_runtime(m, copies, block_bytes, misses_per_layer):
+    """q* recomputed from bandwidths measured in this run: every timed miss copy
+    folded into the PCIe estimate, a host-memory copy into the host estimate."""
+    try:
+        est = m.BandwidthEstimate(alpha=0.25)
+        for ms, n in copies:
+            if ms > 0 and n > 0:
+                est.observe("pcie", n * block_bytes, ms * 1e-3)
+        hb, threads = host_bandwidth_gbs()
+        est.observe("host", hb * 1e9, 1.0)
+        mm = int(round(misses_per_layer))
+        qg, qc, r = est.qstar(mm)
+        return {"b_pcie_gbs": round(est.b_pcie, 2), "b_host_gbs": round(est.b_host, 2),
+                "host_threads": threads, "pcie_observations": int(est.est.n_pcie),
+                "misses_per_layer": mm, "q_gpu": qg, "q_cpu": qc, "ratio": round(r, 4)}
+    except Exception as e:          # a report, never a reason to lose the bench line
+        return {"error": str(e)[:200]}
+
+
 def decode_config(w, T, world):
     """The `config` object of the decode line (both arms)."""
     return {"workload": w.name, "layers": w.L, "batch": T, "format": w.fmt,
@@ -600,6 +641,7 @@ def main():
     xs_host = torch.from_numpy(np.ascontiguousarray(xs[:, :, :T]).view(np.int16)).view(torch.bfloat16).pin_memory()
     e2e = e2e_run(torch, m, w, pool, T, xs_host, wr, bias, args.steps, args.warmup,
                   overlap=not args.no_overlap)
+    pool_block_bytes = pool.block_bytes
     pool.close()
 
     # all-resident pool: the FFN kernel's own HBM roofline on the same layers
@@ -632,6 +674,7 @@ def main():
     h2d_gbs = st["h2d_bytes"] / (copy_ms * 1e-3) / 1e9 if copy_ms > 0 else None
     ratio = profiled_traffic_ratio("ffn_decode_kernel_decode_35b_t1.md", "ffn_decode.cu")
     traffic = int(ratio * alg_avg) if ratio else None
+    qstar_rt = qstar_runtime(m, r["copy"], pool_block_bytes, st["misses"] / max(1, args.steps * w.L))
 
     if rank == 0:
         cb = oracle_sample(w, T, experts, budget_s=args.oracle_budget) if world == 1 else None
@@ -652,6 +695,7 @@ def main():
             "gpu_launches": 4 * w.L * args.steps,
             "clocks": clocks,
             "h2d_gbs": round(h2d_gbs, 2) if h2d_gbs else None,
+            "qstar_runtime": qstar_rt,
             "h2d_bytes_per_step": st["h2d_bytes"] // args.steps,
             "hit_rate": round(st["hits"] / max(1, st["unique"]), 4),
             "misses_per_layer": round(st["misses"] / (args.steps * w.L), 3),

@@ -15,6 +15,7 @@ ERR_NAMES = {1: "MOE_EINVAL", 2: "MOE_ENOMEM", 3: "MOE_ECUDA", 4: "MOE_ETIMEOUT"
              5: "MOE_EBOUNDS", 6: "MOE_ESTATE"}
 MOE_MXFP4, MOE_NVFP4 = 0, 1
 MOE_COPY_SM, MOE_COPY_DMA = 0, 1
+MOE_BW_PCIE, MOE_BW_HOST = 0, 1
 STATUS_READY_TIMEOUT, STATUS_DEP_TIMEOUT, STATUS_BAD_SLOT, STATUS_BAD_EXPERT, STATUS_PIPE_TIMEOUT = 1, 2, 4, 8, 16
 
 
@@ -37,6 +38,11 @@ class Miss(C.Structure):
 class LookupResult(C.Structure):
     _fields_ = [("n_uniq", C.c_int), ("n_miss", C.c_int), ("uniq_h", C.POINTER(C.c_int32)),
                 ("is_hit_h", C.POINTER(C.c_int32)), ("miss_h", C.POINTER(Miss))]
+
+
+class BwEstimate(C.Structure):
+    _fields_ = [("alpha", C.c_double), ("b_pcie", C.c_double), ("b_host", C.c_double),
+                ("n_pcie", C.c_longlong), ("n_host", C.c_longlong)]
 
 
 class Stats(C.Structure):
@@ -75,6 +81,9 @@ SIGNATURES = {
     "moe_decode_layer": (i32, [vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,
                                C.POINTER(LookupResult), vp, vp, i32, vp, vp]),
     "qstar_split": (i32, [i32, f64, f64, C.POINTER(i32), C.POINTER(i32), C.POINTER(f64)]),
+    "moe_bw_init": (i32, [C.POINTER(BwEstimate), f64, f64, f64]),
+    "moe_bw_observe": (i32, [C.POINTER(BwEstimate), i32, f64, f64]),
+    "moe_bw_qstar": (i32, [C.POINTER(BwEstimate), i32, C.POINTER(i32), C.POINTER(i32), C.POINTER(f64)]),
     "moe_dequant_slot": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_set_wait_limits": (i32, [f64, f64, f64]),
     "moe_set_ffn_trace": (i32, [vp]),

@@ -197,6 +197,36 @@ def combine(y_part, y, stream=None):
     L.check("moe_combine", L.load().moe_combine(_p(y_part), T, k, H, _p(y), _s(stream)))
 
 
+class BandwidthEstimate:
+    """Moving estimates of PCIe and host-memory bandwidth (GB/s) and the q* split
+    recomputed from them (moe_bw_init / moe_bw_observe / moe_bw_qstar)."""
+
+    def __init__(self, alpha=0.25, b_pcie=0.0, b_host=0.0):
+        self.est = L.BwEstimate()
+        L.check("moe_bw_init", L.load().moe_bw_init(C.byref(self.est), float(alpha), float(b_pcie),
+                                                     float(b_host)))
+
+    def observe(self, link, nbytes, seconds):
+        """link: "pcie" or "host"."""
+        which = {"pcie": L.MOE_BW_PCIE, "host": L.MOE_BW_HOST}[link]
+        L.check("moe_bw_observe", L.load().moe_bw_observe(C.byref(self.est), which, float(nbytes),
+                                                           float(seconds)))
+
+    @property
+    def b_pcie(self):
+        return self.est.b_pcie
+
+    @property
+    def b_host(self):
+        return self.est.b_host
+
+    def qstar(self, m):
+        qg, qc, r = C.c_int(), C.c_int(), C.c_double()
+        L.check("moe_bw_qstar", L.load().moe_bw_qstar(C.byref(self.est), int(m), C.byref(qg), C.byref(qc),
+                                                       C.byref(r)))
+        return qg.value, qc.value, r.value
+
+
 def qstar_split(m, b_pcie, b_host):
     qg, qc, r = C.c_int(), C.c_int(), C.c_double()
     L.check("qstar_split", L.load().qstar_split(int(m), float(b_pcie), float(b_host),

@@ -311,6 +311,38 @@ extern "C" int moe_pool_set_copy_mode(moe_pool* p, int mode) {
     return MOE_OK;
 }
 
+extern "C" int moe_bw_init(moe_bw_estimate* est, double alpha, double b_pcie0, double b_host0) {
+    if (!est) return fail(MOE_EINVAL, "null estimate");
+    if (!(alpha > 0.0 && alpha <= 1.0) || !(b_pcie0 >= 0.0) || !(b_host0 >= 0.0) || !std::isfinite(b_pcie0) ||
+        !std::isfinite(b_host0))
+        return fail(MOE_EINVAL, "bandwidth estimate: alpha in (0, 1], initial bandwidths finite and >= 0");
+    est->alpha = alpha;
+    est->b_pcie = b_pcie0;
+    est->b_host = b_host0;
+    est->n_pcie = 0;
+    est->n_host = 0;
+    return MOE_OK;
+}
+
+extern "C" int moe_bw_observe(moe_bw_estimate* est, int which, double bytes, double seconds) {
+    if (!est) return fail(MOE_EINVAL, "null estimate");
+    if ((which != MOE_BW_PCIE && which != MOE_BW_HOST) || !(bytes > 0.0) || !(seconds > 0.0) ||
+        !std::isfinite(bytes) || !std::isfinite(seconds))
+        return fail(MOE_EINVAL, "bandwidth observation: link MOE_BW_PCIE/MOE_BW_HOST, bytes and seconds > 0");
+    const double obs = bytes / seconds / 1e9;
+    double& b = which == MOE_BW_PCIE ? est->b_pcie : est->b_host;
+    long long& n = which == MOE_BW_PCIE ? est->n_pcie : est->n_host;
+    b = b > 0.0 ? (1.0 - est->alpha) * b + est->alpha * obs : obs;
+    n += 1;
+    return MOE_OK;
+}
+
+extern "C" int moe_bw_qstar(const moe_bw_estimate* est, int m, int* q_gpu, int* q_cpu, double* ratio) {
+    if (!est) return fail(MOE_EINVAL, "null estimate");
+    if (!(est->b_pcie > 0.0) || !(est->b_host > 0.0)) return fail(MOE_ESTATE, "a bandwidth is not yet known");
+    return qstar_split(m, est->b_pcie, est->b_host, q_gpu, q_cpu, ratio);
+}
+
 extern "C" int qstar_split(int m, double b_pcie, double b_host, int* q_gpu, int* q_cpu, double* ratio) {
     if (!q_gpu || !q_cpu || !ratio) return fail(MOE_EINVAL, "null output");
     if (m < 0 || !(b_pcie > 0.0) || !(b_host > 0.0) || !std::isfinite(b_pcie) || !std::isfinite(b_host))

@@ -334,6 +334,27 @@ int moe_decode_layer(moe_pool* pool, int layer, const void* x_bf16, int T, const
  * Host only.  Errors: MOE_EINVAL (m < 0 or a bandwidth <= 0). */
 int qstar_split(int m, double b_pcie, double b_host, int* q_gpu, int* q_cpu, double* ratio);
 
+/* Run-time bandwidth adaptation of q* (post.smzdm.com/p/a825qpgl section 二: the
+ * split follows the machine's measured PCIe and host-memory bandwidths; "跑不快大
+ * 模型，先别急着怪显卡" section 二: pull : compute = pcie_bw : (cpu_bw - pcie_bw)).
+ * A moving estimate of each bandwidth, fed with observed transfers, from which
+ * q* is recomputed whenever the caller asks (e.g. every step).  Host only. */
+enum { MOE_BW_PCIE = 0, MOE_BW_HOST = 1 };
+typedef struct {
+    double alpha;               /* weight of a new observation, in (0, 1] */
+    double b_pcie, b_host;      /* current estimates in GB/s; 0 = not yet known */
+    long long n_pcie, n_host;   /* observations folded in */
+} moe_bw_estimate;
+/* Reset: alpha in (0, 1]; initial estimates >= 0 (0 = unknown).  MOE_EINVAL. */
+int moe_bw_init(moe_bw_estimate* est, double alpha, double b_pcie0, double b_host0);
+/* Fold one transfer of `bytes` in `seconds` (both > 0) over link `which`:
+ * est = obs if the estimate is unknown, else (1 - alpha) * est + alpha * obs,
+ * obs = bytes / seconds / 1e9.  MOE_EINVAL on bad arguments. */
+int moe_bw_observe(moe_bw_estimate* est, int which, double bytes, double seconds);
+/* qstar_split(m, b_pcie, b_host) of the current estimates; MOE_ESTATE while
+ * either bandwidth is unknown. */
+int moe_bw_qstar(const moe_bw_estimate* est, int m, int* q_gpu, int* q_cpu, double* ratio);
+
 /* Dequantise tensor `which` (0 gate, 1 up, 2 down) of the expert in `slot`
  * to fp32 [rows, K] in canonical order: (e2m1(c) * scale) * S_tensor, two fp32
  * multiplies (the second only for NVFP4).  key = layer*E + expert selects the
