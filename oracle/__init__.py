@@ -58,6 +58,7 @@ def lib():
             "or_lru_create": (vp, [i32, i32]), "or_lru_destroy": (None, [vp]),
             "or_lru_state": (None, [vp, vp, vp, vp, vp]),
             "or_lru_step": (i32, [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
+            "or_lru_resize": (i32, [vp, i32]),
             "or_expert_ffn": (None, [i32, i32, i32, vp, vp, vp]),
             "or_moe_decode": (None, [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
             "or_moe_dense": (None, [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
@@ -183,6 +184,14 @@ class LRU:
         u, m = nu.value, nm.value
         return dict(slot_of=slot_of, uniq=uniq[:u].copy(), hit=hit[:u].astype(bool),
                     miss_expert=me[:m].copy(), miss_slot=ms[:m].copy(), evicted=ev[:m].copy())
+
+    def resize(self, n_new):
+        """Resize to n_new slots; returns the number of evicted entries."""
+        rc = lib().or_lru_resize(self._h, int(n_new))
+        if rc < 0:
+            raise ValueError("n_new must be >= 1")
+        self.n_slots = int(n_new)
+        return rc
 
     def state(self):
         sk = np.empty(self.n_slots, np.int32)

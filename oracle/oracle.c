@@ -312,6 +312,52 @@ void or_lru_state(const or_lru* p, int32_t* slot_key, uint64_t* slot_clock, int3
     *clock = p->clock;
 }
 
+/* Resize the pool to n_new slots (survey's next row: trade slot-pool HBM for a
+ * KV cache at run time without losing the LRU state; reading stated in the
+ * design notes).  Shrinking evicts the residents with the oldest clocks until at
+ * most n_new remain, then moves each survivor that sits in a slot >= n_new, in
+ * ascending slot order, to the lowest free slot below n_new (its clock moves with
+ * it).  Growing adds empty slots.  The global clock is unchanged.  Returns the
+ * number of evictions, or -1 if n_new < 1. */
+int or_lru_resize(or_lru* p, int n_new)
+{
+    if (n_new < 1) return -1;
+    if (n_new > p->n_slots) {
+        p->slot_key = (int32_t*)realloc(p->slot_key, sizeof(int32_t) * (size_t)n_new);
+        p->slot_clock = (uint64_t*)realloc(p->slot_clock, sizeof(uint64_t) * (size_t)n_new);
+        for (int s = p->n_slots; s < n_new; s++) {
+            p->slot_key[s] = -1;
+            p->slot_clock[s] = 0;
+        }
+        p->n_slots = n_new;
+        return 0;
+    }
+    int resident = 0, evicted = 0;
+    for (int s = 0; s < p->n_slots; s++) resident += p->slot_key[s] >= 0;
+    while (resident > n_new) {          /* evict the least recently used */
+        int v = -1;
+        for (int s = 0; s < p->n_slots; s++)
+            if (p->slot_key[s] >= 0 && (v < 0 || p->slot_clock[s] < p->slot_clock[v])) v = s;
+        p->key_slot[p->slot_key[v]] = -1;
+        p->slot_key[v] = -1;
+        p->slot_clock[v] = 0;
+        resident--;
+        evicted++;
+    }
+    int free_slot = 0;
+    for (int s = n_new; s < p->n_slots; s++) {
+        if (p->slot_key[s] < 0) continue;
+        while (p->slot_key[free_slot] >= 0) free_slot++;   /* exists: residents <= n_new */
+        p->slot_key[free_slot] = p->slot_key[s];
+        p->slot_clock[free_slot] = p->slot_clock[s];
+        p->key_slot[p->slot_key[s]] = free_slot;
+        p->slot_key[s] = -1;
+        p->slot_clock[s] = 0;
+    }
+    p->n_slots = n_new;
+    return evicted;
+}
+
 /* One (step, layer) lookup.  Outputs: slot_of[T*k]; uniq[] = sorted unique experts
  * with is_hit[] per entry (returns their count via *n_uniq); miss list
  * miss_expert[], miss_slot[], evicted_key[] (-1 when a free slot was used) in

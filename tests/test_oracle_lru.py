@@ -97,3 +97,60 @@ def test_lru_rejects_pool_smaller_than_step(orc):
     pool = orc.LRU(2, 1, 8)
     with pytest.raises(ValueError):
         pool.step(0, np.array([[0, 1, 2]], np.int32))
+
+
+def _list_resize(ref, n_new):
+    """Textbook resize of a list LRU: keep the n_new most recently used keys."""
+    while len(ref.order) > n_new:
+        ref.order.popitem(last=False)
+    ref.cap = n_new
+
+
+@pytest.mark.parametrize("sizes", [(12, 5, 9, 3, 16), (20, 20, 7, 30), (8, 1, 8)])
+def test_lru_resize_matches_list_lru(orc, sizes):
+    """Resizing keeps the most recently used entries and the LRU order: the slot pool
+    then behaves step for step like a list LRU truncated to its n most recent keys."""
+    L, E, T, k = 2, 24, 1, 1 if min(sizes) < 3 else 3
+    rng = np.random.default_rng(sum(sizes))
+    pool = orc.LRU(sizes[0], L, E)
+    ref = ListLRU(sizes[0])
+    trace = list(_trace(rng, 60 * len(sizes), L, E, T, k, 0.6))
+    for phase, n in enumerate(sizes):
+        if phase:
+            before = list(ref.order)
+            ev = pool.resize(n)
+            _list_resize(ref, n)
+            assert ev == len(before) - len(ref.order)
+            st = pool.state()
+            resident = sorted(q for q in st["slot_key"].tolist() if q >= 0)
+            assert resident == sorted(ref.order) and len(st["slot_key"]) == n
+            # the clocks keep the list order of the survivors
+            by_clock = [st["slot_key"][s] for s in np.argsort(st["slot_clock"]) if st["slot_key"][s] >= 0]
+            assert by_clock == list(ref.order)
+            for s, q in enumerate(st["slot_key"].tolist()):
+                if q >= 0:
+                    assert st["key_slot"][q] == s
+        for layer, idx in trace[phase * 60:(phase + 1) * 60]:
+            r = pool.step(layer, idx)
+            keys = [layer * E + e for e in r["uniq"].tolist()]
+            hits, misses, victims = ref.step(keys)
+            assert [layer * E + e for e, h in zip(r["uniq"], r["hit"]) if h] == hits
+            assert r["evicted"].tolist() == victims
+
+
+def test_lru_resize_moves_survivors_to_lowest_free_slots(orc):
+    pool = orc.LRU(6, 1, 8)
+    for e in range(6):                                   # expert e in slot e, clock e + 1
+        pool.step(0, np.array([[e]], np.int32))
+    pool.step(0, np.array([[1]], np.int32))              # expert 1 -> clock 7 (most recent)
+    assert pool.resize(3) == 3                           # evicts clocks 1, 3, 4: experts 0, 2, 3
+    st = pool.state()
+    # survivors 1 (slot 1), 4 (slot 4 -> 0), 5 (slot 5 -> 2)
+    assert st["slot_key"].tolist() == [4, 1, 5]
+    assert st["slot_clock"].tolist() == [5, 7, 6] and st["clock"] == 7
+    assert pool.resize(5) == 0
+    assert pool.state()["slot_key"].tolist() == [4, 1, 5, -1, -1]
+    r = pool.step(0, np.array([[6]], np.int32))          # a fresh slot, the lowest free one
+    assert r["miss_slot"].tolist() == [3] and r["evicted"].tolist() == [-1]
+    with pytest.raises(ValueError):
+        pool.resize(0)
