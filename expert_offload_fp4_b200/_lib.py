@@ -76,6 +76,8 @@ SIGNATURES = {
     "moe_slot_lookup_result": (i32, [vp, C.POINTER(LookupResult)]),
     "moe_stream_misses": (i32, [vp, i32, C.POINTER(Miss), i32, vp]),
     "moe_pool_set_copy_mode": (i32, [vp, i32]),
+    "moe_pool_resize": (i32, [vp, i32]),
+    "moe_lru_plan_resize": (i32, [vp, vp, i32, i32, vp, C.POINTER(i32), vp, vp, C.POINTER(i32)]),
     "moe_expert_ffn": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp]),
     "moe_combine": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_decode_layer": (i32, [vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,

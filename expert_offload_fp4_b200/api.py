@@ -39,6 +39,7 @@ class Pool:
         self.cfg = L.MoeConfig(H, I, E, k, L_layers, FMT[fmt], n_slots, max_tokens, host_layers)
         self.H, self.I, self.E, self.k, self.L = H, I, E, k, L_layers
         self.fmt, self.n_slots, self.max_tokens = fmt, n_slots, max_tokens
+        self.n_active = n_slots
         self.host_layers = host_layers or L_layers
         h = C.c_void_p()
         L.check("moe_pool_create", self.lib.moe_pool_create(C.byref(self.cfg), C.byref(h)))
@@ -76,6 +77,11 @@ class Pool:
         n = self.n_slots if n_active_slots is None else int(n_active_slots)
         L.check("moe_pool_reset", self.lib.moe_pool_reset(self.handle, n))
         self.n_active = n
+
+    def resize(self, n_active_slots):
+        """Resize the slot pool at run time, keeping the LRU state (moe_pool_resize)."""
+        L.check("moe_pool_resize", self.lib.moe_pool_resize(self.handle, int(n_active_slots)))
+        self.n_active = int(n_active_slots)
 
     def set_copy_mode(self, mode):
         """"sm" (a kernel reads the mapped host block over PCIe) or "dma" (copy engine)."""
@@ -195,6 +201,20 @@ def decode_layer(pool, layer, x, wr, bias, renormalize, idx, w, slot_of, y_part,
 def combine(y_part, y, stream=None):
     T, k, H = y_part.shape
     L.check("moe_combine", L.load().moe_combine(_p(y_part), T, k, H, _p(y), _s(stream)))
+
+
+def lru_plan_resize(slot_key, slot_clock, n_new):
+    """moe_lru_plan_resize on host arrays: (evicted slots, [(from, to) moves])."""
+    sk = np.ascontiguousarray(slot_key, np.int32)
+    sc = np.ascontiguousarray(slot_clock, np.uint64)
+    n_old = len(sk)
+    ev, mf, mt = (np.zeros(n_old, np.int32) for _ in range(3))
+    ne, nm = C.c_int(), C.c_int()
+    L.check("moe_lru_plan_resize", L.load().moe_lru_plan_resize(
+        sk.ctypes.data_as(C.c_void_p), sc.ctypes.data_as(C.c_void_p), n_old, int(n_new),
+        ev.ctypes.data_as(C.c_void_p), C.byref(ne), mf.ctypes.data_as(C.c_void_p),
+        mt.ctypes.data_as(C.c_void_p), C.byref(nm)))
+    return ev[:ne.value].tolist(), list(zip(mf[:nm.value].tolist(), mt[:nm.value].tolist()))
 
 
 class BandwidthEstimate:

@@ -5,6 +5,8 @@
 #include <cmath>
 #include <string>
 
+#include <vector>
+
 #include "common.cuh"
 
 namespace moe {
@@ -240,6 +242,97 @@ extern "C" int moe_pool_reset(moe_pool* p, int n_active_slots) {
     MOE_CUDA_TRY(cudaMemset(p->ready, 0, S * sizeof(uint32_t)));
     p->n_active = n_active_slots;
     memset(&p->stats, 0, sizeof(p->stats));
+    return MOE_OK;
+}
+
+extern "C" int moe_lru_plan_resize(const int32_t* slot_key_h, const uint64_t* slot_clock_h, int n_old, int n_new,
+                                   int32_t* evict_slot_h, int* n_evict, int32_t* move_from_h, int32_t* move_to_h,
+                                   int* n_move) {
+    if (!slot_key_h || !slot_clock_h || !evict_slot_h || !n_evict || !move_from_h || !move_to_h || !n_move)
+        return fail(MOE_EINVAL, "null argument");
+    if (n_old < 1 || n_new < 1) return fail(MOE_EINVAL, "resize plan: slot counts must be >= 1");
+    *n_evict = 0;
+    *n_move = 0;
+    if (n_new >= n_old) return MOE_OK;                   // growing: new slots start empty
+    // residents ordered by last touch, oldest first; the oldest go until n_new remain
+    std::vector<std::pair<uint64_t, int>> res;
+    for (int s = 0; s < n_old; s++)
+        if (slot_key_h[s] >= 0) res.push_back({slot_clock_h[s], s});
+    std::sort(res.begin(), res.end());
+    const int drop = std::max(0, (int)res.size() - n_new);
+    std::vector<char> gone(n_old, 0);
+    for (int i = 0; i < drop; i++) {
+        evict_slot_h[(*n_evict)++] = res[i].second;
+        gone[res[i].second] = 1;
+    }
+    // survivors above the new end, in slot order, into the lowest free slots below it
+    int dst = 0;
+    for (int s = n_new; s < n_old; s++) {
+        if (slot_key_h[s] < 0 || gone[s]) continue;
+        while (dst < n_new && slot_key_h[dst] >= 0 && !gone[dst]) dst++;
+        if (dst >= n_new) return fail(MOE_ESTATE, "resize plan: no free slot (inconsistent state)");
+        move_from_h[*n_move] = s;
+        move_to_h[*n_move] = dst;
+        (*n_move)++;
+        dst++;
+    }
+    return MOE_OK;
+}
+
+extern "C" int moe_pool_resize(moe_pool* p, int n_new) {
+    if (!p) return fail(MOE_EINVAL, "null pool");
+    if (n_new < 1 || n_new > p->cfg.n_slots) return fail(MOE_EINVAL, "resize: active slots must be in [1, n_slots]");
+    if (p->lk_pending) return fail(MOE_ESTATE, "resize: a launched lookup has not been collected");
+    const int S = p->cfg.n_slots, n_old = p->n_active;
+    const size_t LE = size_t(p->cfg.L) * p->cfg.E;
+    MOE_CUDA_TRY(cudaDeviceSynchronize());
+    std::vector<int32_t> sk(S), ks(LE);
+    std::vector<uint64_t> sc(S);
+    std::vector<uint32_t> need(S), ready(S);
+    MOE_CUDA_TRY(cudaMemcpy(sk.data(), p->slot_key, S * 4, cudaMemcpyDeviceToHost));
+    MOE_CUDA_TRY(cudaMemcpy(sc.data(), p->slot_clock, S * 8, cudaMemcpyDeviceToHost));
+    MOE_CUDA_TRY(cudaMemcpy(ks.data(), p->key_slot, LE * 4, cudaMemcpyDeviceToHost));
+    MOE_CUDA_TRY(cudaMemcpy(need.data(), p->need, S * 4, cudaMemcpyDeviceToHost));
+    MOE_CUDA_TRY(cudaMemcpy(ready.data(), p->ready, S * 4, cudaMemcpyDeviceToHost));
+    // an entry whose copy never landed holds no expert: drop it first
+    for (int s = 0; s < n_old; s++)
+        if (sk[s] >= 0 && ready[s] != need[s]) {
+            ks[sk[s]] = -1;
+            sk[s] = -1;
+            sc[s] = 0;
+        }
+    std::vector<int32_t> ev(S), mf(S), mt(S);
+    int ne = 0, nm = 0;
+    int rc = moe_lru_plan_resize(sk.data(), sc.data(), n_old, n_new, ev.data(), &ne, mf.data(), mt.data(), &nm);
+    if (rc) return rc;
+    for (int i = 0; i < ne; i++) {
+        const int s = ev[i];
+        ks[sk[s]] = -1;
+        sk[s] = -1;
+        sc[s] = 0;
+    }
+    for (int i = 0; i < nm; i++) {
+        const int from = mf[i], to = mt[i];
+        MOE_CUDA_TRY(cudaMemcpy(p->slots + size_t(to) * p->lay.bytes, p->slots + size_t(from) * p->lay.bytes,
+                                p->lay.bytes, cudaMemcpyDeviceToDevice));
+        sk[to] = sk[from];
+        sc[to] = sc[from];
+        ks[sk[to]] = to;
+        need[to] = ready[to] = need[from];   // the block is present: its ticket is published
+        sk[from] = -1;
+        sc[from] = 0;
+    }
+    for (int s = std::min(n_old, n_new); s < S; s++) {   // slots outside the active range are empty
+        sk[s] = -1;
+        sc[s] = 0;
+    }
+    MOE_CUDA_TRY(cudaMemcpy(p->slot_key, sk.data(), S * 4, cudaMemcpyHostToDevice));
+    MOE_CUDA_TRY(cudaMemcpy(p->slot_clock, sc.data(), S * 8, cudaMemcpyHostToDevice));
+    MOE_CUDA_TRY(cudaMemcpy(p->key_slot, ks.data(), LE * 4, cudaMemcpyHostToDevice));
+    MOE_CUDA_TRY(cudaMemcpy(p->need, need.data(), S * 4, cudaMemcpyHostToDevice));
+    MOE_CUDA_TRY(cudaMemcpy(p->ready, ready.data(), S * 4, cudaMemcpyHostToDevice));
+    p->n_active = n_new;
+    p->stats.evictions += ne;
     return MOE_OK;
 }
 

@@ -144,6 +144,26 @@ int moe_pool_reset(moe_pool* pool, int n_active_slots);
 /* Copy the LRU state to host arrays (synchronous; for checks and checkpoints):
  * slot_key_h[n_slots] (layer*E+expert or -1), slot_clock_h[n_slots],
  * key_slot_h[L*E] (slot or -1), *clock_h = global clock. */
+/* Resize the slot pool to n_active_slots in [1, n_slots] at run time, keeping the
+ * LRU state (to trade slot-pool HBM for other memory, e.g. a KV cache): shrinking
+ * evicts the residents with the oldest clocks until at most n_active_slots remain
+ * and moves every survivor sitting above the new end, in slot order, to the
+ * lowest free slot below it (a device-to-device copy of its block; its clock and
+ * ready ticket move with it); growing adds empty slots.  Entries whose copy never
+ * landed (ready ticket != needed ticket) are dropped first.  The global clock is
+ * unchanged, so later lookups continue the same LRU order.  Synchronises the
+ * device: call between steps with no pool work in flight.  Errors: MOE_EINVAL,
+ * MOE_ESTATE (a launched lookup not collected), MOE_ECUDA. */
+int moe_pool_resize(moe_pool* pool, int n_active_slots);
+
+/* The resize decision on host copies of the first n_old slots' state (for
+ * checks): evict_slot_h receives the evicted slots (oldest clock first),
+ * move_from_h / move_to_h the moves, in order.  Arrays hold n_old entries.
+ * Errors: MOE_EINVAL, MOE_ESTATE (inconsistent state). */
+int moe_lru_plan_resize(const int32_t* slot_key_h, const uint64_t* slot_clock_h, int n_old, int n_new,
+                        int32_t* evict_slot_h, int* n_evict, int32_t* move_from_h, int32_t* move_to_h,
+                        int* n_move);
+
 int moe_pool_read_state(moe_pool* pool, int32_t* slot_key_h, uint64_t* slot_clock_h,
                         int32_t* key_slot_h, uint64_t* clock_h);
 int moe_pool_stats(const moe_pool* pool, moe_stats* out);

@@ -441,6 +441,53 @@ def test_copy_modes_fill_slots_identically(m, mode):
     pool.close()
 
 
+def test_pool_resize_keeps_lru_state_and_outputs(m):
+    """Shrink and grow a live pool between steps: the slot table follows the
+    oracle's resize bit for bit (moved blocks included) and later layers still
+    match the oracle."""
+    w = small("rs", "mxfp4", H=256, I=256, E=16, k=2, L=2, zipf=0.7)
+    T = 2
+    pool = m.Pool(w.H, w.I, w.E, w.k, w.L, w.fmt, 12, max_tokens=T)
+    for layer in range(w.L):
+        for e in range(w.E):
+            pool.load_expert(layer, e, weights(w, layer, e))
+    ref = oracle.LRU(12, w.L, w.E)
+    lo = m.DecodeLayer(pool, T)
+
+    def steps(s0, n):
+        for step in range(s0, s0 + n):
+            for layer in range(w.L):
+                x = gen.activations(w, layer, step, T)
+                wr = gen.router_weight(w, layer)
+                b = gen.router_bias(w, layer)
+                lo(layer, bf16(x), bf16(wr), dev(b))
+                torch.cuda.synchronize()
+                check_layer(w, lo, x, wr, b, layer)
+                r = ref.step(layer, lo.idx.cpu().numpy())
+                assert [s for _, s, _, _ in lo.lookup.miss_list()] == r["miss_slot"].tolist()
+
+    def same_state(n_active):
+        got, want = pool.read_state(), ref.state()
+        assert got["slot_key"][:n_active].tolist() == want["slot_key"].tolist()
+        assert (got["slot_key"][n_active:] < 0).all()
+        assert got["slot_clock"][:n_active].tolist() == want["slot_clock"].tolist()
+        assert np.array_equal(got["key_slot"], want["key_slot"]) and got["clock"] == want["clock"]
+
+    steps(0, 4)
+    same_state(12)
+    pool.resize(5)
+    ref.resize(5)
+    same_state(5)
+    steps(4, 3)
+    same_state(5)
+    pool.resize(12)
+    ref.resize(12)
+    same_state(12)
+    steps(7, 2)
+    same_state(12)
+    pool.close()
+
+
 def test_pool_reset_restricts_active_slots(m):
     """After a reset to n active slots the LRU behaves as a fresh n-slot pool."""
     E, k, L = 32, 4, 2
