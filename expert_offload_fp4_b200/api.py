@@ -188,7 +188,9 @@ def decode_layer(pool, layer, x, wr, bias, renormalize, idx, w, slot_of, y_part,
                  lookup=None, copy_events=None, overlap=True, stream=None, copy_stream=None):
     """moe_decode_layer: route, lookup, FFN, miss copies and combine of one layer."""
     T = x.shape[0]
-    cs = copy_stream if copy_stream is not None else stream
+    if copy_stream is None:
+        raise ValueError("decode_layer needs a copy_stream of its own (torch.cuda.Stream())")
+    cs = copy_stream
     ev0, ev1 = (None, None) if copy_events is None else (C.c_void_p(copy_events[0].cuda_event),
                                                         C.c_void_p(copy_events[1].cuda_event))
     L.check("moe_decode_layer", pool.lib.moe_decode_layer(

@@ -18,6 +18,9 @@ extern "C" int moe_decode_layer(moe_pool* p, int layer, const void* x_bf16, int 
                                 void* copy_start, void* copy_end, int overlap, void* stream,
                                 void* copy_stream) {
     if (!p) return fail(MOE_EINVAL, "null pool");
+    // with overlap the FFN waits for copies issued after it: they need their own stream
+    if (overlap && (copy_stream == stream || copy_stream == nullptr))
+        return fail(MOE_EINVAL, "decode layer: copy_stream must be a stream other than the compute stream");
     const moe_config& c = p->cfg;
     // the caller's result arrays, else local ones of the largest size a call needs
     int32_t uniq_l[kMaxE], hit_l[kMaxE];

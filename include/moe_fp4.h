@@ -338,7 +338,9 @@ int moe_combine(const float* y_part, int T, int k, int H, void* y_bf16, void* st
  * status (device int); route_ws of moe_route_workspace_bytes(T, E) bytes.
  * res: host arrays that receive the lookup result (capacity >= min(T*k, E)),
  * or NULL.  copy_start / copy_end: CUDA events recorded on copy_stream before
- * and after the miss copies when the layer has misses, or NULL.  overlap = 0
+ * and after the miss copies when the layer has misses, or NULL.  With overlap,
+ * copy_stream must be a non-blocking stream other than `stream` (the FFN waits for
+ * copies issued after it; MOE_EINVAL if it is the same stream or NULL).  overlap = 0
  * waits for the miss list and issues the copies before the FFN is enqueued
  * (for tools that serialise kernels).  Returns the first failing call's error;
  * a launched lookup is collected even when the FFN launch fails. */

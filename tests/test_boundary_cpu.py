@@ -95,4 +95,10 @@ def test_route_argument_checks_need_no_gpu(lib):
     assert L.moe_decode_layer(None, 0, p, 1, p, None, 1, p, p, p, p, p, p, p, 64, None, None, None, 1,
                               None, None) == lib.MOE_EINVAL
     assert L.moe_pool_set_copy_mode(None, lib.MOE_COPY_DMA) == lib.MOE_EINVAL
+    # with overlap, a copy stream equal to the compute stream would deadlock: refused
+    fake_pool = C.c_void_p(p.value)
+    s1 = C.c_void_p(0x1000)
+    assert L.moe_decode_layer(fake_pool, 0, p, 1, p, None, 1, p, p, p, p, p, p, p, 64, None, None, None, 1,
+                              s1, s1) == lib.MOE_EINVAL
+    assert b"copy_stream" in L.moe_last_error()
     assert L.moe_set_wait_limits(-1.0, 1.0, 1.0) == lib.MOE_EINVAL
