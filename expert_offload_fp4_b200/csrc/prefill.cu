@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(256) prefill_quant_kernel(const uint16_t* __re
                                                            int E, const int32_t* __restrict__ idx, PrefillWs ws,
                                                            uint8_t* __restrict__ out_codes,
                                                            uint8_t* __restrict__ out_scales,
-                                                           float* __restrict__ out_sx, float* __restrict__ y0) {
+                                                           float* __restrict__ out_sx) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (warp >= T) return;
     const int t = warp;
@@ -194,10 +194,6 @@ __global__ void __launch_bounds__(256) prefill_quant_kernel(const uint16_t* __re
             for (int i = 0; i < 4; i++)
                 amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[i] << 16)), fabsf(__uint_as_float(w4[i] & 0xFFFF0000u))));
         }
-    }
-    if (y0) {   // the down GEMM accumulates into y: zero this token's row here
-        float4* yr = reinterpret_cast<float4*>(y0 + (size_t)t * H);
-        for (int v = lane; v < H / 4; v += 32) yr[v] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -549,7 +545,7 @@ extern "C" int moe_nvfp4_quantize(const void* x_bf16, int T, int H, uint8_t* cod
     PrefillWs ws{};
     const int blocks = (T * 32 + 255) / 256;
     prefill_quant_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>((const uint16_t*)x_bf16, T, H, 0, 0, nullptr, ws,
-                                                                   codes, scales, sx, nullptr);
+                                                                   codes, scales, sx);
     MOE_CUDA_TRY(cudaGetLastError());
     return MOE_OK;
 }
@@ -593,7 +589,7 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
     prefill_plan_kernel<<<1, 1024, 0, s>>>(idx, slot_of, T * c.k, c.E, ws, status);
     MOE_CUDA_TRY(cudaGetLastError());
     prefill_quant_kernel<<<(T * 32 + 255) / 256, 256, 0, s>>>((const uint16_t*)x_bf16, T, c.H, c.k, c.E, idx, ws,
-                                                              nullptr, nullptr, nullptr, y);
+                                                              nullptr, nullptr, nullptr);
     MOE_CUDA_TRY(cudaGetLastError());
 
     const size_t pool_bytes = size_t(c.n_slots) * B.bytes;
@@ -631,6 +627,9 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
     const int grid1 = std::min(PL.MT * g.NT, p->num_sms);
     grouped_gemm_kernel<1><<<grid1, kPThreads, smem, s>>>(ma1, msa1, mb1, msb1, g);
     MOE_CUDA_TRY(cudaGetLastError());
+    // y is zeroed only now, after GEMM1 has streamed its weights through L2, so that
+    // the down GEMM's reductions into it find it in L2
+    MOE_CUDA_TRY(cudaMemsetAsync(y, 0, size_t(T) * c.H * sizeof(float), s));
     // GEMM2 reads the down rows of the slot with its own pitch
     g.b_rows_per_slot = B.bytes / dr;
     g.b_sf_rows_per_slot = B.bytes / ds;
