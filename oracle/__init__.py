@@ -3,7 +3,9 @@
 TEST INFRASTRUCTURE: only the tests, the smoke check and the benchmark's
 CPU-baseline leg import this package.  It never touches the CUDA library.
 Functions here only marshal numpy arrays into the C calls; all arithmetic is in
-oracle.c.
+oracle.c, except in prefill_batch.py, which runs the prefill path's per-token
+dot products of oracle.c as float64 matrix products (a library matmul as one
+step) so that a whole 2048-token prompt can be checked in seconds.
 """
 from __future__ import annotations
 
@@ -63,6 +65,7 @@ def lib():
             "or_moe_decode": (None, [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
             "or_moe_dense": (None, [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
             "or_moe_prefill_token": (None, [i32, i32, i32, vp, vp, vp, vp, vp, vp]),
+            "or_prefill_h_rows": (None, [vp, vp, i32, i32, vp, vp]),
             "or_qstar_split": (i32, [i32, f64, f64, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
@@ -268,6 +271,17 @@ def moe_prefill_token(H, I, E, x_t, idx_t, w_t, experts: dict):
     lib().or_moe_prefill_token(H, I, idx_t.shape[0], _p(x_t), _p(idx_t), _p(w_t), arr,
                                _p(yf), _p(yb))
     return yf, yb
+
+
+def prefill_h_rows(g, u):
+    """h = fp32(silu(g) * u) of [rows, I] double dot products, quantised to NVFP4
+    with tensor scale 1: (codes [rows, I/2], scales [rows, I/16])."""
+    g, u = _c(g, np.float64), _c(u, np.float64)
+    rows, I = g.shape
+    codes = np.empty((rows, I // 2), np.uint8)
+    scales = np.empty((rows, I // 16), np.uint8)
+    lib().or_prefill_h_rows(_p(g), _p(u), rows, I, _p(codes), _p(scales))
+    return codes, scales
 
 
 # ------------------------------------------------------------------------------- q*

@@ -312,9 +312,10 @@ void or_lru_state(const or_lru* p, int32_t* slot_key, uint64_t* slot_clock, int3
     *clock = p->clock;
 }
 
-/* Resize the pool to n_new slots (survey's next row: trade slot-pool HBM for a
- * KV cache at run time without losing the LRU state; reading stated in the
- * design notes).  Shrinking evicts the residents with the oldest clocks until at
+/* Resize the pool to n_new slots (post.smzdm.com/p/aomxznrn, "FreeToken干的事":
+ * at run time the engine moves GPU memory between the expert cache and the KV
+ * cache; read here as shrinking or growing the slot pool while keeping the LRU
+ * order of what stays).  Shrinking evicts the residents with the oldest clocks until at
  * most n_new remain, then moves each survivor that sits in a slot >= n_new, in
  * ascending slot order, to the lowest free slot below n_new (its clock moves with
  * it).  Growing adds empty slots.  The global clock is unchanged.  Returns the
@@ -583,6 +584,22 @@ void or_moe_prefill_token(int H, int I, int k, const uint16_t* x_t, const int32_
     free(xq); free(xc); free(xs);
     free(hf); free(hq); free(hc); free(hs);
     free(acc);
+}
+
+/* The h step of the prefill path for many rows at once: for every row r of the
+ * [rows, I] double gate and up dot products, h = (float)(silu(g) * u), quantised
+ * to NVFP4 with tensor scale 1 (the same steps as inside or_moe_prefill_token).
+ * Writes codes [rows, I/2] and scales [rows, I/16]. */
+void or_prefill_h_rows(const double* g, const double* u, int rows, int I, uint8_t* codes,
+                       uint8_t* scales)
+{
+    float* hf = (float*)malloc(sizeof(float) * (size_t)I);
+    for (int r = 0; r < rows; r++) {
+        for (int i = 0; i < I; i++)
+            hf[i] = (float)(silu(g[(size_t)r * I + i]) * u[(size_t)r * I + i]);
+        or_nvfp4_quantize_row(hf, I, 1.0f, codes + (size_t)r * (I / 2), scales + (size_t)r * (I / 16));
+    }
+    free(hf);
 }
 
 /* ------------------------------------------------------------------------ q* [q*] */

@@ -181,3 +181,25 @@ def test_prefill_x_quantisation_is_exact_on_grid_at_any_scale(orc, k):
     assert S == np.float32(2.0 ** (k - 10))
     assert np.all(s == 0x7E)                             # 448 in every block
     assert np.array_equal(orc.dequant("nvfp4", c[None], s[None], S)[0], x)
+
+
+def test_batched_prefill_equals_per_token_oracle(orc):
+    """oracle.prefill_batch (float64 matrix products over every token of an
+    expert) against or_moe_prefill_token (plain per-token loops) on uneven groups:
+    both take the same steps, only the order of the float64 additions inside a
+    dot product differs, so they agree to float64 rounding.  A transposed weight,
+    a wrong rank order or a dropped routing weight moves the output by O(rms)."""
+    from oracle import prefill_batch
+    w = W.Workload(name="pb", H=256, I=256, E=8, k=3, L=1, fmt=W.NVFP4, seed=31, batches=(40,),
+                   steps=1, zipf_s=0.9, weight_recipe="normal")
+    T = 40
+    x = gen.activations(w, 0, 0, T)
+    idx, wt, _ = orc.route(x, gen.router_weight(w, 0), gen.router_bias(w, 0), w.k, 1)
+    experts = {e: gen.expert_weights(w, 0, e) for e in range(w.E)}
+    yb = prefill_batch.moe_prefill(w.H, w.I, w.E, x, idx, wt, experts)
+    counts = np.bincount(idx.ravel(), minlength=w.E)
+    assert counts.min() != counts.max()            # the groups really are uneven
+    for t in range(T):
+        yt, _ = orc.moe_prefill_token(w.H, w.I, w.E, x[t], idx[t], wt[t], experts)
+        rms = float(np.sqrt(np.mean(yt.astype(np.float64) ** 2)))
+        assert float(np.max(np.abs(yb[t] - yt))) <= 1e-5 * rms, t
