@@ -180,6 +180,7 @@ def ffn_roofline(torch, m, w, pool, T, x_dev, wr, bias, reps=4):
     wt = torch.empty((L_, T, w.k), dtype=torch.float32, device="cuda")
     slot_of = torch.empty((L_, T, w.k), dtype=torch.int32, device="cuda")
     y_part = torch.empty((T, w.k, w.H), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, w.H), dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     ws = torch.zeros(m.route_workspace_bytes(T, w.E), dtype=torch.uint8, device="cuda")
     uniq = []
@@ -189,7 +190,7 @@ def ffn_roofline(torch, m, w, pool, T, x_dev, wr, bias, reps=4):
         assert res.n_miss == 0, "roofline pass expects an all-resident pool"
         uniq.append(res.n_uniq)
     for l in range(L_):     # warm-up
-        m.expert_ffn(pool, l, x_dev[l], idx[l], wt[l], slot_of[l], y_part, status)
+        m.expert_ffn(pool, l, x_dev[l], idx[l], wt[l], slot_of[l], y_part, status, y=y)
     torch.cuda.synchronize()
     cur = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -197,7 +198,7 @@ def ffn_roofline(torch, m, w, pool, T, x_dev, wr, bias, reps=4):
     e0.record(cur)
     for r in range(reps):
         for l in range(L_):
-            m.expert_ffn(pool, l, x_dev[l], idx[l], wt[l], slot_of[l], y_part, status)
+            m.expert_ffn(pool, l, x_dev[l], idx[l], wt[l], slot_of[l], y_part, status, y=y)
     e1.record(cur)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
@@ -209,6 +210,12 @@ def expert_bytes_alg(w):
     """Algorithmic HBM bytes of one expert: FP4 codes + block scales of gate, up, down."""
     bs = W.block_elems(w.fmt)
     return 3 * (w.H * w.I // 2 + w.H * w.I // bs)
+
+
+def ffn_alg_bytes(w, T, uniq):
+    """Algorithmic HBM bytes of one decode FFN launch with the fused combine: the
+    weights of the unique experts, x in, y_part [T, k, H] fp32 and y [T, H] bf16 out."""
+    return uniq * expert_bytes_alg(w) + T * w.H * 2 + T * w.k * w.H * 4 + T * w.H * 2
 
 
 # ---------------------------------------------------------------- ranks
@@ -318,7 +325,9 @@ def oracle_sample(w, T, experts, budget_s=10.0, min_layers=2):
 
 
 def ffn_only(args, w, T):
-    """The decode FFN kernel alone on `args.layers` all-resident layer positions."""
+    """The decode FFN kernel alone on `args.layers` all-resident layer positions;
+    --trace adds per-CTA phase stamps (median and max over CTAs, us from the
+    earliest CTA start)."""
     from dataclasses import replace
     wl = replace(w, L=args.layers)
     experts = gen.expert_weights_many(wl, 0, range(wl.E))
@@ -331,27 +340,35 @@ def ffn_only(args, w, T):
     wr = torch.from_numpy(gen.router_weight(wl, 0).view(np.int16)).cuda().view(torch.bfloat16)
     bias = torch.from_numpy(gen.router_bias(wl, 0)).cuda()
     ms, uniq = ffn_roofline(torch, m, wl, pool, T, x_dev, wr, bias, reps=2)
+    info = m.ffn_launch_info(pool, T)
     phases = None
     if args.trace:
-        buf = torch.zeros((148, 64), dtype=torch.int64, device="cuda")
-        m._lib.load().moe_set_ffn_trace(buf.data_ptr())
+        buf = torch.zeros((148 * 2, 32), dtype=torch.int64, device="cuda")
+        m._lib.load().moe_set_ffn_trace(C_ptr(buf))
         ffn_roofline(torch, m, wl, pool, T, x_dev, wr, bias, reps=1)
         m._lib.load().moe_set_ffn_trace(None)
-        tr = buf.cpu().numpy().astype(np.float64)
+        tr = buf.cpu().numpy()
+        n_cta = info["cluster"] * info["clusters"]
+        tr = tr[:n_cta].astype(np.float64)
         t0 = tr[:, 0].min()
-        rel = (tr[:, :8] - t0) / 1000.0
-        if args.trace_out:
-            np.save(args.trace_out, buf.cpu().numpy())
-        phases = {name: [round(float(np.median(rel[:, i])), 2), round(float(rel[:, i].max()), 2)]
-                  for i, name in enumerate(["start", "lookup_done", "table", "first_data", "a_done",
-                                            "b_dep", "items_done", "end"])}
+        names = ["start", "staged", "pdl", "table", "first_data", "a_done", "published", "gathered",
+                 "b_done", "counted", "end", "last_copy"]
+        phases = {nm: [round(float(np.median(tr[:, i] - t0)) / 1e3, 2), round(float((tr[:, i] - t0).max()) / 1e3, 2)]
+                  for i, nm in enumerate(names)}
+        phases["groups_per_cta_max"] = int(tr[:, 12].max())
+        phases["stage_landed"] = [round(float(np.median(tr[:, 16 + i] - t0)) / 1e3, 2) for i in range(8)]
+        phases["stage_issued"] = [round(float(np.median(tr[:, 24 + i] - t0)) / 1e3, 2) for i in range(8)]
     pool.close()
-    per = expert_bytes_alg(wl)
-    alg = sum(u * per + T * wl.H * 2 + T * wl.k * wl.H * 4 for u in uniq) / len(uniq)
+    alg = sum(ffn_alg_bytes(wl, T, u) for u in uniq) / len(uniq)
     print(json.dumps({"mode": "ffn", "workload": wl.name, "layers": wl.L, "batch": T,
                       "launch_ms_avg": round(ms, 5), "alg_bytes_per_launch": int(alg),
-                      "achieved_gbs": round(alg / (ms * 1e-3) / 1e9, 1),
+                      "achieved_gbs": round(alg / (ms * 1e-3) / 1e9, 1), "launch": info,
                       "phases_us_median_max": phases}), flush=True)
+
+
+def C_ptr(t):
+    import ctypes
+    return ctypes.c_void_p(t.data_ptr())
 
 
 # ------------------------------------------------------- 284B decode + cache stress
@@ -542,8 +559,7 @@ def main():
                     help="ffn: only the decode FFN kernel on a small all-resident pool "
                          "(a few layers), e.g. for an ncu capture")
     ap.add_argument("--layers", type=int, default=4, help="layer positions in --mode ffn")
-    ap.add_argument("--trace", action="store_true", help="--mode ffn: per-CTA phase timestamps")
-    ap.add_argument("--trace-out", default="", help="--trace: also save the raw stamps (.npy)")
+    ap.add_argument("--trace", action="store_true", help="--mode ffn: per-CTA phase stamps")
     ap.add_argument("--host-layers", type=int, default=8,
                     help="--mode offload: distinct host copies of the 40 layers (pinned RAM)")
     ap.add_argument("--no-overlap", action="store_true",
@@ -653,7 +669,7 @@ def main():
     ffn_ms, ffn_u = ffn_roofline(torch, m, w, rpool, T, xd[0], wr, bias)
     rpool.close()
     per_exp = expert_bytes_alg(w)
-    alg_bytes = [u * per_exp + T * w.H * 2 + T * w.k * w.H * 4 for u in ffn_u]
+    alg_bytes = [ffn_alg_bytes(w, T, u) for u in ffn_u]
     alg_avg = sum(alg_bytes) / len(alg_bytes)
     achieved = alg_avg / (ffn_ms * 1e-3) / 1e9
 

@@ -78,7 +78,10 @@ SIGNATURES = {
     "moe_pool_set_copy_mode": (i32, [vp, i32]),
     "moe_pool_resize": (i32, [vp, i32]),
     "moe_lru_plan_resize": (i32, [vp, vp, i32, i32, vp, C.POINTER(i32), vp, vp, C.POINTER(i32)]),
-    "moe_expert_ffn": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp]),
+    "moe_set_ffn_trace": (i32, [vp]),
+    "moe_set_ffn_cluster": (i32, [i32]),
+    "moe_ffn_launch_info": (i32, [vp, i32, vp, vp, vp, vp]),
+    "moe_expert_ffn": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp]),
     "moe_combine": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_decode_layer": (i32, [vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,
                                C.POINTER(LookupResult), vp, vp, i32, vp, vp]),
@@ -88,7 +91,6 @@ SIGNATURES = {
     "moe_bw_qstar": (i32, [C.POINTER(BwEstimate), i32, C.POINTER(i32), C.POINTER(i32), C.POINTER(f64)]),
     "moe_dequant_slot": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_set_wait_limits": (i32, [f64, f64, f64]),
-    "moe_set_ffn_trace": (i32, [vp]),
     "moe_nvfp4_gemm": (i32, [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]),
     "moe_nvfp4_quantize": (i32, [vp, i32, i32, vp, vp, vp, vp]),
     "moe_prefill_workspace_bytes": (sz, [vp, i32]),

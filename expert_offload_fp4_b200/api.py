@@ -177,11 +177,25 @@ def stream_misses(pool, layer, lookup, copy_stream):
         pool.handle, int(layer), lookup.misses, lookup.res.n_miss, _s(copy_stream)))
 
 
-def expert_ffn(pool, layer, x, idx, w, slot_of, y_part, status, stream=None):
+def expert_ffn(pool, layer, x, idx, w, slot_of, y_part, status, y=None, stream=None):
+    """moe_expert_ffn: y_part [T, k, H] fp32; with y [T, H] bf16 also the fused combine."""
     T = x.shape[0]
     L.check("moe_expert_ffn", pool.lib.moe_expert_ffn(
-        pool.handle, int(layer), _p(x), T, _p(idx), _p(w), _p(slot_of), _p(y_part), _p(status),
+        pool.handle, int(layer), _p(x), T, _p(idx), _p(w), _p(slot_of), _p(y_part), _p(y), _p(status),
         _s(stream)))
+
+
+def set_ffn_cluster(cluster):
+    """moe_set_ffn_cluster: CTAs per expert of later decode FFN launches (0 = automatic)."""
+    L.check("moe_set_ffn_cluster", L.load().moe_set_ffn_cluster(int(cluster)))
+
+
+def ffn_launch_info(pool, T):
+    """moe_ffn_launch_info: the decode FFN's launch shape for T tokens on this pool."""
+    c, n, st, sm = C.c_int(), C.c_int(), C.c_int(), C.c_int()
+    L.check("moe_ffn_launch_info", pool.lib.moe_ffn_launch_info(
+        pool.handle, int(T), C.byref(c), C.byref(n), C.byref(st), C.byref(sm)))
+    return dict(cluster=c.value, clusters=n.value, stages=st.value, smem_bytes=sm.value)
 
 
 def decode_layer(pool, layer, x, wr, bias, renormalize, idx, w, slot_of, y_part, y, status, ws,

@@ -96,14 +96,17 @@ struct moe_pool {
     int lk_seq;                   // sequence number of the last launched lookup
     int lk_pending;               // a launched lookup whose record was not collected
     int lk_attr_set;
-    // decode FFN scratch
-    float* hbuf;                  // [kMaxDecodePairs][I] fp32
-    unsigned int* hamax;          // [kMaxDecodePairs] |h| max as float bits
-    unsigned int* ctr;            // [kMaxDecodePairs] h rows done per group, then done + abort
+    // decode FFN counters: [0, 16) groups done per row block (the fused combine),
+    // then the abort flag and the count of finished CTAs
+    unsigned int* ctr;
     // copy engine ready-flag write
     void* write_value32;          // cuStreamWriteValue32 entry point
-    int ffn_attr_set[2][5];       // decode FFN launch attributes set, per (format, token bucket)
-    int ffn_per_sm[2][5];
+    int ffn_attr_set[2][2];       // decode FFN launch attributes set, per (format, token tiles)
+    int ffn_ncl[2][2][5];         // clusters of 16, 8, 4, 2, 1 CTAs that fit on the GPU at once
+                                  // (0: that size does not split the pool's shapes)
+    CUtensorMap ffn_map_a[2];     // gate/up code rows, boxes of 16 / 32 rows
+    CUtensorMap ffn_map_b[4];     // down code rows, boxes of 16 / 32 / 64 / 128 rows
+    int ffn_map_a_ok[2], ffn_map_b_ok[4];
     moe_stats stats;
 };
 

@@ -6,7 +6,7 @@
 // on the GPU while missing ones cross PCIe): router and lookup are enqueued,
 // then the FFN, whose CTAs on resident experts start at once; only then does
 // the host wait (bounded) for the lookup's miss list and put the misses on the
-// copy stream; the combine follows the FFN on the compute stream.
+// copy stream.  The combine is fused into the FFN kernel.
 #include "common.cuh"
 
 using namespace moe;
@@ -43,15 +43,13 @@ extern "C" int moe_decode_layer(moe_pool* p, int layer, const void* x_bf16, int 
         // misses streamed before the FFN is enqueued (for tools that serialise kernels)
         if ((rc = moe_slot_lookup(p, layer, idx, T, c.k, slot_of, r, stream))) return rc;
         if ((rc = copies())) return rc;
-        if ((rc = moe_expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, status, stream))) return rc;
-        return moe_combine(y_part, T, c.k, c.H, y_bf16, stream);
+        return moe_expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, y_bf16, status, stream);
     }
     if ((rc = moe_slot_lookup_launch(p, layer, idx, T, c.k, slot_of, stream))) return rc;
-    rc = moe_expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, status, stream);
+    rc = moe_expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, y_bf16, status, stream);
     // the launched lookup is collected whatever the FFN launch returned
     const int rc2 = moe_slot_lookup_result(p, r);
     if (rc) return rc;
     if (rc2) return rc2;
-    if ((rc = copies())) return rc;
-    return moe_combine(y_part, T, c.k, c.H, y_bf16, stream);
+    return copies();
 }

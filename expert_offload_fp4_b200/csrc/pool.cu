@@ -86,8 +86,6 @@ extern "C" int moe_pool_destroy(moe_pool* p) {
     cudaFree(p->need);
     cudaFree(p->ready);
     cudaFree(p->tscale);
-    cudaFree(p->hbuf);
-    cudaFree(p->hamax);
     cudaFree(p->ctr);
     if (p->host) cudaFreeHost(p->host);
     if (p->lk_h) cudaFreeHost(p->lk_h);
@@ -137,8 +135,6 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
     ALLOC(p->need, S * sizeof(uint32_t));
     ALLOC(p->ready, S * sizeof(uint32_t));
     ALLOC(p->tscale, LE * 3 * sizeof(float));
-    ALLOC(p->hbuf, size_t(kMaxDecodePairs) * cfg->I * sizeof(float));
-    ALLOC(p->hamax, kMaxDecodePairs * sizeof(unsigned int));
     ALLOC(p->ctr, (kMaxDecodePairs + 8) * sizeof(unsigned int));
 #undef ALLOC
     cudaMemset(p->slot_key, 0xFF, S * sizeof(int32_t));
@@ -149,7 +145,6 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
     cudaMemset(p->need, 0, S * sizeof(uint32_t));
     cudaMemset(p->ready, 0, S * sizeof(uint32_t));
     cudaMemset(p->tscale, 0, LE * 3 * sizeof(float));
-    cudaMemset(p->hamax, 0, kMaxDecodePairs * sizeof(unsigned int));
     cudaMemset(p->ctr, 0, (kMaxDecodePairs + 8) * sizeof(unsigned int));
     e = cudaHostAlloc((void**)&p->host, host_bytes, cudaHostAllocMapped);
     if (e != cudaSuccess) {

@@ -1,5 +1,5 @@
 """One decode MoE layer through the C ABI: route -> slot lookup -> miss
-streaming (copy stream) -> expert FFN (compute stream) -> combine.
+streaming (copy stream) -> expert FFN with the combine fused in (compute stream).
 
 This is the public call a user makes per (token batch, layer); it owns only the
 per-call device buffers.  The copy of missed experts runs on its own stream and
@@ -76,15 +76,15 @@ class DecodeLayer:
             api.slot_lookup(p, layer, self.idx, self.slot_of, self.lookup, stream)
             if self.lookup.n_miss:
                 api.stream_misses(p, layer, self.lookup, self.copy_stream)
-            api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, stream)
-            api.combine(self.y_part, self.y, stream)
+            api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, self.y,
+                           stream)
             return self.y
         api.slot_lookup_launch(p, layer, self.idx, self.slot_of, stream)
         if self.ffn_events is not None:
             cur = stream if stream is not None else torch.cuda.current_stream()
             fe = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             fe[0].record(cur)
-        api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, stream)
+        api.expert_ffn(p, layer, x, self.idx, self.w, self.slot_of, self.y_part, self.status, self.y, stream)
         if self.ffn_events is not None:
             fe[1].record(cur)
         # nothing that can wait for the device between the FFN launch and the copies
@@ -97,7 +97,6 @@ class DecodeLayer:
             if self.copy_events is not None:
                 ev[1].record(self.copy_stream)
                 self.copy_events.append((ev, self.lookup.n_miss))
-        api.combine(self.y_part, self.y, stream)
         if self.ffn_events is not None:
             self.ffn_events.append((fe, self.lookup.n_uniq, self.lookup.n_miss))
         return self.y

@@ -63,7 +63,7 @@ enum {
 /* Bits of the device status word written by moe_expert_ffn. */
 enum {
     MOE_STATUS_READY_TIMEOUT = 1,  /* a missed expert's ready flag never arrived */
-    MOE_STATUS_DEP_TIMEOUT = 2,    /* down projection waited too long for h */
+    MOE_STATUS_DEP_TIMEOUT = 2,    /* waited too long for the cluster's slices of h */
     MOE_STATUS_BAD_SLOT = 4,       /* slot index outside the pool */
     MOE_STATUS_BAD_EXPERT = 8,     /* expert index outside [0, E) */
     MOE_STATUS_PIPE_TIMEOUT = 16   /* a shared-memory pipeline wait gave up */
@@ -244,44 +244,65 @@ int moe_stream_misses(moe_pool* pool, int layer, const moe_miss* miss_h, int n_m
  * registers and shared memory for that).  Errors: MOE_EINVAL. */
 int moe_pool_set_copy_mode(moe_pool* pool, int mode);
 
-/* Decode expert FFN (post.smzdm.com/p/aomxznrn: decode is bandwidth-bound and
- * scheduled apart from prefill).  For every (t, j): y_part[t, j, :] =
- * w[t,j] * Wd (silu(Wg x_t) * (Wu x_t)) of expert idx[t,j] read from slot
- * slot_of[t,j]; FP4 weights dequantised on the fly (MXFP4: e2m1 * 2^(s-127);
- * NVFP4: e2m1 * e4m3(s) * S_tensor): exact f16 products summed in f16 within a
- * scale block, block sums scaled and accumulated in fp32, h rounded to f16 with a
- * per-token power-of-two scale.  One persistent kernel, one CTA per SM, fed by
- * bulk copies into a shared-memory ring; its CTAs wait on one another (down rows
- * need all gate/up rows of their expert) and on the ready tickets of missed
- * experts.  It is a plain launch with programmatic stream serialisation: it
- * stages x while the kernel before it (the slot lookup) finishes.  Waits are
- * bounded (moe_set_wait_limits) and failures set bits of *status (device int,
- * caller-zeroed; MOE_STATUS_*): if other work keeps one of its CTAs off the GPU
- * for longer than the limits, the call reports a timeout instead of hanging.
- * y_part is [T, k, H] fp32.  Limits: T <= max_tokens of the pool.
+/* Decode expert FFN (post.smzdm.com/p/aomxznrn, "FreeToken干的事": decode is
+ * bandwidth-bound and scheduled apart from prefill; post.smzdm.com/p/a825qpgl
+ * section 二: expert results merged by routing weight).  For every (t, j):
+ * y_part[t, j, :] = w[t,j] * Wd (silu(Wg x_t) * (Wu x_t)) of expert idx[t,j] read
+ * from slot slot_of[t,j]; FP4 weights dequantised on the fly (MXFP4: e2m1 *
+ * 2^(s-127); NVFP4: e2m1 * e4m3(s) * S_tensor).  Arithmetic: every product of a
+ * weight and an activation is exact and the sums are fp32 (tensor-core MMA with
+ * fp32 accumulation); x enters as f16 after a per-token power of two (exact for
+ * bf16 x down to 2^-24 of the token's largest element), h as the sum of two f16
+ * values (about 22 significant bits).  If y_bf16 is not NULL the call also does
+ * the combine: y_bf16[t, :] = bf16(sum over j = 0..k-1 of y_part[t, j, :]),
+ * summed in fp32 in rank order, round to nearest even (the same as moe_combine).
+ * One thread-block cluster per unique expert computes it (gate/up rows split
+ * over the cluster's CTAs, h exchanged through distributed shared memory, down
+ * rows split again); CTAs wait only for CTAs of their own cluster and for the
+ * ready tickets of missed experts.  It is a plain launch with programmatic
+ * stream serialisation: it stages x while the kernel before it (the slot lookup)
+ * finishes, so x must be complete before that kernel starts (it is, when the
+ * router ran on x first).  Waits are bounded (moe_set_wait_limits); failures set
+ * bits of *status (device int, caller-zeroed; MOE_STATUS_*).  y_part is [T, k, H]
+ * fp32, y_bf16 [T, H]; x, y_part and y_bf16 16-byte aligned.  Limits: T <=
+ * max_tokens of the pool, and T * (H + 2 I) * 2 bytes of activations must fit in
+ * shared memory beside two weight stages (MOE_EINVAL otherwise).
  * Errors: MOE_EINVAL. */
 int moe_expert_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const int32_t* idx,
-                   const float* w, const int32_t* slot_of, float* y_part, int* status,
+                   const float* w, const int32_t* slot_of, float* y_part, void* y_bf16, int* status,
                    void* stream);
 
 /* Limits of the device-side bounded waits of moe_expert_ffn, in milliseconds:
- * a missed expert's ready flag (default 5000), the down projection's wait for
- * all rows of h (default 5000), a shared-memory pipeline stage (default 10000).
+ * a missed expert's ready flag (default 5000), the wait for the other CTAs of
+ * a cluster to publish their slices of h (default 5000), a shared-memory
+ * pipeline stage (default 10000).
  * Process-wide; affects later launches.  Errors: MOE_EINVAL (non-positive). */
 int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
 
-/* Tracing: when buf is a device buffer of at least 64 * 148 (64 per SM) u64,
- * each CTA of every later moe_expert_ffn launch writes global-timer stamps (ns)
- * at row blockIdx * 64: [0] start, [1] the preceding kernel (the slot lookup)
- * complete and the activations staged, [2] expert table built,
- * [3] first item's weights landed, [4] gate/up items done and published,
- * [5] first down item's h dependency met, [6] last item done, [7] end;
- * for the CTA's first 16 items j: [8 + 2j] its weights landed (first consumer
- * warp), [9 + 2j] that warp done with it, [40 + j] its copies issued; [56] the
- * CTA's item count and [57] how many of them are gate/up items (counts, not
- * times); SM clock counts (clock64) for its item 1 on the first consumer warp:
- * [62] weights landed, [58] dot products start, [59] dot products done,
- * [60] lane reductions done, [61] epilogue done, [63] stage released.  Unwritten entries keep their old value.  NULL turns tracing off. */
+/* Cluster size of later moe_expert_ffn launches (for tuning sweeps): 1, 2, 4,
+ * 8 or 16 CTAs per expert where the shapes and the GPU allow it (otherwise the
+ * automatic choice), 0 = automatic (the default: the size with the least work
+ * per CTA counting the rounds in which the clusters take the experts).
+ * Process-wide.  Errors: MOE_EINVAL. */
+int moe_set_ffn_cluster(int cluster);
+
+/* Launch shape moe_expert_ffn uses on this pool for T tokens (for reports):
+ * CTAs per cluster, clusters launched, shared-memory weight stages per CTA,
+ * dynamic shared memory per CTA in bytes.  Errors: MOE_EINVAL. */
+int moe_ffn_launch_info(moe_pool* pool, int T, int* cluster, int* clusters, int* nstage, int* smem_bytes);
+
+/* Tracing (for profiling): when buf is a device buffer of at least 32 u64 per
+ * CTA of the largest launch (32 * 296 covers every launch), each CTA of every
+ * later moe_expert_ffn launch writes, at row blockIdx * 32, global-timer stamps
+ * in ns: [0] start, [1] activations staged and the cluster started,
+ * [2] the preceding kernel (the slot lookup) complete, [3] group table built,
+ * [4] first weights landed, [5] first group's slice of h done, [6] the cluster's
+ * slices published, [7] whole h gathered, [8] first group's down rows done,
+ * [9] last group counted (and combined), [10] end, [11] the producer's last copy
+ * issued, [16 + s] stage s of the first group landed (consumer side, s < 8),
+ * [24 + s] the producer's copies of its s-th stage issued (s < 8); and counts:
+ * [12] groups of the CTA, [13] CTAs per cluster, [14] rank in the cluster.
+ * Unwritten entries keep their old value.  NULL turns tracing off. */
 int moe_set_ffn_trace(void* buf);
 
 /* Block-scaled NVFP4 GEMM on the tcgen05 tensor cores (the contraction of
@@ -331,9 +352,9 @@ int moe_combine(const float* y_part, int T, int k, int H, void* y_bf16, void* st
 /* One decode MoE layer in one call (the engine's per-layer sequence,
  * post.smzdm.com/p/aomxznrn "FreeToken干的事": resident experts compute on the
  * GPU while missing ones cross PCIe).  Runs moe_route, moe_slot_lookup_launch,
- * moe_expert_ffn, moe_slot_lookup_result (the one host wait, bounded),
- * moe_stream_misses on copy_stream and moe_combine, with the arguments and
- * rules of those calls; k, H and E come from the pool.  Caller-owned device
+ * moe_expert_ffn with the combine fused in (y_bf16), moe_slot_lookup_result (the
+ * one host wait, bounded) and moe_stream_misses on copy_stream, with the
+ * arguments and rules of those calls; k, H and E come from the pool.  Caller-owned device
  * buffers: idx, w, slot_of [T, k]; y_part [T, k, H] fp32; y_bf16 [T, H];
  * status (device int); route_ws of moe_route_workspace_bytes(T, E) bytes.
  * res: host arrays that receive the lookup result (capacity >= min(T*k, E)),
