@@ -335,6 +335,7 @@ def ffn_only(args, w, T):
     import expert_offload_fp4_b200 as m
     pool = make_pool(m, wl, wl.L * wl.E, 8, 1, experts)
     preload(torch, m, pool, wl)
+    m.set_ffn_cluster(args.ffn_cluster)
     xs = np.stack([gen.activations(wl, l, 0, T) for l in range(wl.L)])
     x_dev = torch.from_numpy(xs.view(np.int16)).cuda().view(torch.bfloat16)
     wr = torch.from_numpy(gen.router_weight(wl, 0).view(np.int16)).cuda().view(torch.bfloat16)
@@ -559,6 +560,8 @@ def main():
                     help="ffn: only the decode FFN kernel on a small all-resident pool "
                          "(a few layers), e.g. for an ncu capture")
     ap.add_argument("--layers", type=int, default=4, help="layer positions in --mode ffn")
+    ap.add_argument("--ffn-cluster", type=int, default=0,
+                    help="--mode ffn: force the decode FFN's cluster size (0: automatic)")
     ap.add_argument("--trace", action="store_true", help="--mode ffn: per-CTA phase stamps")
     ap.add_argument("--host-layers", type=int, default=8,
                     help="--mode offload: distinct host copies of the 40 layers (pinned RAM)")

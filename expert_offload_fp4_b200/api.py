@@ -185,7 +185,7 @@ def expert_ffn(pool, layer, x, idx, w, slot_of, y_part, status, y=None, stream=N
         _s(stream)))
 
 
-def set_ffn_cluster(cluster):
+def set_ffn_cluster(cluster=0):
     """moe_set_ffn_cluster: CTAs per expert of later decode FFN launches (0 = automatic)."""
     L.check("moe_set_ffn_cluster", L.load().moe_set_ffn_cluster(int(cluster)))
 

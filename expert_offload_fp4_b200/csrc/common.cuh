@@ -104,9 +104,6 @@ struct moe_pool {
     int ffn_attr_set[2][2];       // decode FFN launch attributes set, per (format, token tiles)
     int ffn_ncl[2][2][5];         // clusters of 16, 8, 4, 2, 1 CTAs that fit on the GPU at once
                                   // (0: that size does not split the pool's shapes)
-    CUtensorMap ffn_map_a[2];     // gate/up code rows, boxes of 16 / 32 rows
-    CUtensorMap ffn_map_b[4];     // down code rows, boxes of 16 / 32 / 64 / 128 rows
-    int ffn_map_a_ok[2], ffn_map_b_ok[4];
     moe_stats stats;
 };
 

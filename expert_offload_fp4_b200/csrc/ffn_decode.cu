@@ -17,24 +17,24 @@
 // y_part over the ranks in rank order and writes the bf16 output rows (K5).
 //
 // Warp specialisation: warp 8 (the producer) streams the FP4 code rows and
-// block scales of each work stage with 1-D bulk copies into a ring of
-// shared-memory stages (mbarrier full/empty pairs; code rows padded so that the
-// consumers' 16-byte reads are bank-conflict free); for a missed expert it first
-// waits (bounded) for the slot's ready ticket written by the copy stream.
+// block scales of each work stage with 1-D bulk copies (a whole tile of rows is
+// one contiguous range of the slot) into a ring of shared-memory stages
+// (mbarrier full/empty pairs); for a missed expert it first waits (bounded) for
+// the slot's ready ticket written by the copy stream.
 // Warps 0..7 (consumers) run the dot products on the tensor cores with
 // mma.sync m16n8k16, f16 inputs and fp32 accumulation:
-//  - weights: E2M1 codes decoded by integer ops to exact f16 values e2m1*2^-14,
+//  - weights: E2M1 code pairs converted to f16 pairs (cvt.rn.f16x2.e2m1x2),
 //    multiplied (exactly) by their block scale in f16: the E4M3 scale itself
 //    (NVFP4), or 2^(e - E) with E the largest E8M0 exponent of the row's
 //    128-element segment (MXFP4; 2^(E-127) is applied to the segment's fp32 sum);
 //  - activations: x of each token times a power of two (bf16 is exact in f16
 //    that way); h of each (token, expert) times a power of two and split into
 //    an f16 high part and an f16 remainder, so down h is carried to ~22 bits;
-//  - products are exact, sums fp32; the K ranges of the 8 warps are added in
-//    warp order, so results are reproducible.
+//  - products are exact, sums fp32; every output row is one warp's chain of
+//    MMAs over the whole K, in a fixed order, so results are reproducible.
 #include <math.h>
 
-#include "tcgen05.cuh"
+#include "common.cuh"
 
 namespace moe {
 
@@ -61,9 +61,6 @@ struct Group {
 };
 
 struct FfnArgs {
-    // the pool's FP4 code rows as 2-D byte tensors (gate/up rows of H/2 bytes, down
-    // rows of I/2), read in boxes 128 bytes wide with the 128-byte swizzle
-    CUtensorMap map_a, map_b;
     const uint16_t* x;
     const int32_t* idx;
     const float* w;
@@ -82,9 +79,10 @@ struct FfnArgs {
     int C;                     // CTAs per cluster
     int RA;                    // gate (and up) rows per A stage: 16 or 32
     int RB;                    // down rows per B stage: 16, 32, 64 or 128
-    int rows_a, rows_b;        // map rows per slot block (block bytes / row bytes)
-    int row_gate, row_up, row_down;   // map row of each tensor's first row inside a block
     int stage_bytes, nstage;
+    int ks;                    // A: K split of a unit (1, 2, 4): 2 ks warps per unit
+    int nAU;                   // A: units at work (divides nstage)
+    int nBU;                   // B: warp groups at work (divides nstage)
     // byte offsets in dynamic shared memory
     int o_groups, o_misc, o_red, o_hloc, o_x, o_h, o_stage;
     unsigned long long ready_ns, dep_ns, pipe_ns;
@@ -127,28 +125,20 @@ __device__ __forceinline__ uint32_t f16_pow2(int d) {
     return 0u;
 }
 
-// Eight values of one 16-byte piece (elements 0..7) as the f16x2 words of the
-// fragment order (0,4), (2,6), (1,5), (3,7): the pairing decode_e2m1_x2 makes.
+// Eight values of one 16-byte piece (elements 0..7) as the f16x2 words (0,1),
+// (2,3), (4,5), (6,7): the pairs a code word's four bytes decode to.
 __device__ __forceinline__ uint4 pack_piece(const float (&f)[8]) {
-    const __half2 w0 = __floats2half2_rn(f[0], f[4]), w1 = __floats2half2_rn(f[2], f[6]);
-    const __half2 w2 = __floats2half2_rn(f[1], f[5]), w3 = __floats2half2_rn(f[3], f[7]);
+    const __half2 w0 = __floats2half2_rn(f[0], f[1]), w1 = __floats2half2_rn(f[2], f[3]);
+    const __half2 w2 = __floats2half2_rn(f[4], f[5]), w3 = __floats2half2_rn(f[6], f[7]);
     return make_uint4(*reinterpret_cast<const uint32_t*>(&w0), *reinterpret_cast<const uint32_t*>(&w1),
                       *reinterpret_cast<const uint32_t*>(&w2), *reinterpret_cast<const uint32_t*>(&w3));
 }
 
-// 8 E2M1 codes (one 32-bit word, element n in bits 4n..4n+3) to 4 f16x2 words,
-// each value e2m1 * 2^-14 exactly: a code's magnitude bits go to f16 bits 11..9
-// (exponent low bits and the top mantissa bit) and its sign to bit 15, so 2^-14
-// scales every value, the E2M1 subnormal 0.5 included.  The f16 high bytes of
-// the even elements (low nibbles) and of the odd ones are formed four at a time;
-// byte moves then give the words (e0,e4), (e2,e6), (e1,e5), (e3,e7).
-__device__ __forceinline__ void decode_word(uint32_t x, uint32_t& w0, uint32_t& w1, uint32_t& w2, uint32_t& w3) {
-    const uint32_t ev = ((x << 1) & 0x0E0E0E0Eu) | ((x << 4) & 0x80808080u);   // bytes: e0 e2 e4 e6
-    const uint32_t od = ((x >> 3) & 0x0E0E0E0Eu) | (x & 0x80808080u);          // bytes: e1 e3 e5 e7
-    w0 = __byte_perm(ev, 0u, 0x2404);
-    w1 = ev & 0xFF00FF00u;
-    w2 = __byte_perm(od, 0u, 0x2404);
-    w3 = od & 0xFF00FF00u;
+// Two E2M1 codes (the low nibble of v's low byte first) -> their f16 values.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t v) {
+    uint32_t h2;
+    asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"(v));
+    return h2;
 }
 
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
@@ -161,8 +151,8 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 // (2 words), D fp32 (4 values).
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    // no side effects: the compiler may interleave independent MMAs
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -256,106 +246,131 @@ __device__ __forceinline__ bool wait_ready(const uint32_t* ready, uint32_t want,
 
 // ------------------------------------------------------------------ tile math
 //
-// One 128-element K segment of TT 16-row tiles against NB B operands of NT
-// 8-column tiles.  Thread (g = lane/4, q = lane%4) reads the 16 code bytes
-// [64 s + 16 q, +16) of rows g and g+8 (elements 32q .. 32q+31 of the segment):
-// word j of them feeds MMA k-tiles 2j and 2j+1.  Inside a k-tile the slots
-// (2q, 2q+1, 2q+8, 2q+9) hold the elements (8j + p, 8j + 4 + p, 8j + 2 + p,
-// 8j + 6 + p) of the thread's 32 (p = 0 for tile 2j, 1 for 2j+1): a fixed
-// permutation of K that the B operands are stored in (see pack_piece), so the
-// products and their sums are those of the plain dot product.
+// The dot products of one 16-row tile with NB B operands of NT 8-column tiles,
+// over the nseg 128-element K segments seg0 .. seg0+nseg-1.  Thread (g = lane/4,
+// q = lane%4) reads the 16 code bytes [64 s + 16 q, +16) of rows g and g+8 of
+// segment s (its elements 32q .. 32q+31): word j of them holds elements
+// 8j .. 8j+7, whose four byte pairs become the A fragments of two MMA k-tiles
+// (k slots 2q, 2q+1 take pair 0 / 2 of the word, slots 2q+8, 2q+9 pair 1 / 3).
+// The B operands are stored in the same order.
 // B operand layout (16-byte pieces): piece (s, j, n, q) holds column n's
-// elements 128 s + 32 q + 8 j + {0,4,2,6,1,5,3,7} at index ((4 s + j) * N + n) * 4 + q;
-// bptr points at (s, 0, n, q) and bstride = 4 N pieces separates the j.
-template <int FMT, int TT, int NT, int NB>
-__device__ __forceinline__ void seg_mma(const uint8_t* const (&code)[TT], uint32_t row8_code,
-                                        const uint8_t* const (&scl)[TT], uint32_t row8_scl, int q,
-                                        const uint4* const (&bptr)[NB][NT], int bstride,
-                                        float (&acc)[TT][NT][4]) {
-    uint4 c[TT], c8[TT];
-    uint32_t fa[TT], fb[TT], fa8[TT], fb8[TT];
-    float post[TT], post8[TT];
+// elements 128 s + 32 q + 8 j + 0..7 at index ((4 s + j) * N + n) * 4 + q;
+// bcol[b][n] points at (0, 0, n, q) (null past the group's columns) and
+// bstride = 4 N pieces separates consecutive j.
+// The two k-tiles of a word and the NB operands go to 2 NB separate fp32
+// accumulators (independent MMA chains), summed in a fixed order at the end;
+// the next segment's codes and scales are loaded before this one is decoded.
+template <int FMT, int NT, int NB>
+__device__ __forceinline__ void tile_mma(const uint8_t* code, uint32_t row8_code, const uint8_t* scl,
+                                         uint32_t row8_scl, int q, int seg0, int nseg,
+                                         const uint4* const (&bcol)[NB][NT], int bstride,
+                                         float (&out)[NT][4]) {
+    constexpr int NA = 2 * NB;
+    constexpr uint32_t sstep = FMT == MOE_NVFP4 ? 8u : 4u;     // scale bytes of a row's segment
+    float acc[NA][NT][4];
 #pragma unroll
-    for (int t = 0; t < TT; t++) {
-        c[t] = *reinterpret_cast<const uint4*>(code[t]);
-        c8[t] = *reinterpret_cast<const uint4*>(code[t] + row8_code);
+    for (int i = 0; i < NA; i++)
+#pragma unroll
+        for (int n = 0; n < NT; n++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) acc[i][n][e] = 0.0f;
+    auto ld_scale = [](const uint8_t* p) -> uint32_t {
+        return FMT == MOE_NVFP4 ? (uint32_t)*reinterpret_cast<const uint16_t*>(p)
+                                : *reinterpret_cast<const uint32_t*>(p);
+    };
+    code += (size_t)seg0 * 64;
+    scl += (size_t)seg0 * sstep;
+    uint4 c = *reinterpret_cast<const uint4*>(code), c8 = *reinterpret_cast<const uint4*>(code + row8_code);
+    uint32_t u = ld_scale(scl), u8 = ld_scale(scl + row8_scl);
+    for (int i = 0; i < nseg; i++) {
+        const int seg = seg0 + i;
+        // the next segment's words (this one's again on the last, in bounds)
+        const uint8_t* cn = code + (i + 1 < nseg ? 64 : 0);
+        const uint8_t* sn = scl + (i + 1 < nseg ? sstep : 0u);
+        const uint4 c_n = *reinterpret_cast<const uint4*>(cn), c8_n = *reinterpret_cast<const uint4*>(cn + row8_code);
+        const uint32_t u_n = ld_scale(sn), u8_n = ld_scale(sn + row8_scl);
+        uint32_t fa, fb, fa8, fb8;
+        float post = 1.0f, post8 = 1.0f;
         if (FMT == MOE_NVFP4) {
             // the thread's two scales per row (blocks 2q, 2q+1 of the segment), exact in f16
-            const uint32_t s = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(scl[t]));
-            const uint32_t s8 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(scl[t] + row8_scl));
-            fa[t] = __byte_perm(s, 0u, 0x1010);
-            fb[t] = __byte_perm(s, 0u, 0x3232);
-            fa8[t] = __byte_perm(s8, 0u, 0x1010);
-            fb8[t] = __byte_perm(s8, 0u, 0x3232);
+            const uint32_t s2 = e4m3x2_to_f16x2(u), s28 = e4m3x2_to_f16x2(u8);
+            fa = __byte_perm(s2, 0u, 0x1010);
+            fb = __byte_perm(s2, 0u, 0x3232);
+            fa8 = __byte_perm(s28, 0u, 0x1010);
+            fb8 = __byte_perm(s28, 0u, 0x3232);
         } else {
             // the 4 E8M0 exponents of the segment; the thread's block (q) relative to their max
-            const uint32_t u = *reinterpret_cast<const uint32_t*>(scl[t]);
-            const uint32_t u8 = *reinterpret_cast<const uint32_t*>(scl[t] + row8_scl);
             uint32_t m = __vmaxu4(u, u >> 8), m8 = __vmaxu4(u8, u8 >> 8);
             m = __vmaxu4(m, m >> 16) & 0xFFu;
             m8 = __vmaxu4(m8, m8 >> 16) & 0xFFu;
             const uint32_t f = f16_pow2((int)((u >> (8 * q)) & 0xFFu) - (int)m);
             const uint32_t f8 = f16_pow2((int)((u8 >> (8 * q)) & 0xFFu) - (int)m8);
-            fa[t] = fb[t] = f | (f << 16);
-            fa8[t] = fb8[t] = f8 | (f8 << 16);
-            post[t] = e8m0_to_f32(m);
-            post8[t] = e8m0_to_f32(m8);
+            fa = fb = f | (f << 16);
+            fa8 = fb8 = f8 | (f8 << 16);
+            post = e8m0_to_f32(m);
+            post8 = e8m0_to_f32(m8);
         }
-    }
-    float sacc[TT][NT][4];
-    if (FMT == MOE_MXFP4) {
+        float sacc[NA][NT][4];     // MXFP4: this segment's sums, before 2^(E-127)
+        if (FMT == MOE_MXFP4) {
 #pragma unroll
-        for (int t = 0; t < TT; t++)
+            for (int a = 0; a < NA; a++)
 #pragma unroll
-            for (int n = 0; n < NT; n++)
+                for (int n = 0; n < NT; n++)
 #pragma unroll
-                for (int e = 0; e < 4; e++) sacc[t][n][e] = 0.0f;
-    }
+                    for (int e = 0; e < 4; e++) sacc[a][n][e] = 0.0f;
+        }
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
-        uint4 bv[NB][NT];
+        for (int j = 0; j < 4; j++) {
+            uint4 bv[NB][NT];
 #pragma unroll
-        for (int b = 0; b < NB; b++)
+            for (int b = 0; b < NB; b++)
 #pragma unroll
-            for (int n = 0; n < NT; n++)
-                bv[b][n] = bptr[b][n] ? bptr[b][n][j * bstride] : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int t = 0; t < TT; t++) {
-            const uint32_t cw = j == 0 ? c[t].x : j == 1 ? c[t].y : j == 2 ? c[t].z : c[t].w;
-            const uint32_t cw8 = j == 0 ? c8[t].x : j == 1 ? c8[t].y : j == 2 ? c8[t].z : c8[t].w;
-            uint32_t r0, r1, r2, r3, s0, s1, s2, s3;
-            decode_word(cw, r0, r1, r2, r3);
-            decode_word(cw8, s0, s1, s2, s3);
-            const uint32_t f = j < 2 ? fa[t] : fb[t], f8 = j < 2 ? fa8[t] : fb8[t];
-            r0 = hmul2_u32(r0, f);
-            r1 = hmul2_u32(r1, f);
-            r2 = hmul2_u32(r2, f);
-            r3 = hmul2_u32(r3, f);
-            s0 = hmul2_u32(s0, f8);
-            s1 = hmul2_u32(s1, f8);
-            s2 = hmul2_u32(s2, f8);
-            s3 = hmul2_u32(s3, f8);
+                for (int n = 0; n < NT; n++)
+                    bv[b][n] = bcol[b][n] ? bcol[b][n][(seg * 4 + j) * bstride] : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t cw = j == 0 ? c.x : j == 1 ? c.y : j == 2 ? c.z : c.w;
+            const uint32_t cw8 = j == 0 ? c8.x : j == 1 ? c8.y : j == 2 ? c8.z : c8.w;
+            const uint32_t f = j < 2 ? fa : fb, f8 = j < 2 ? fa8 : fb8;
+            const uint32_t p0 = hmul2_u32(e2m1x2_to_f16x2(cw), f), p1 = hmul2_u32(e2m1x2_to_f16x2(cw >> 8), f);
+            const uint32_t p2 = hmul2_u32(e2m1x2_to_f16x2(cw >> 16), f), p3 = hmul2_u32(e2m1x2_to_f16x2(cw >> 24), f);
+            const uint32_t t0 = hmul2_u32(e2m1x2_to_f16x2(cw8), f8), t1 = hmul2_u32(e2m1x2_to_f16x2(cw8 >> 8), f8);
+            const uint32_t t2 = hmul2_u32(e2m1x2_to_f16x2(cw8 >> 16), f8), t3 = hmul2_u32(e2m1x2_to_f16x2(cw8 >> 24), f8);
 #pragma unroll
             for (int n = 0; n < NT; n++)
 #pragma unroll
                 for (int b = 0; b < NB; b++) {
-                    float (&d)[4] = FMT == MOE_MXFP4 ? sacc[t][n] : acc[t][n];
-                    mma16816(d, r0, s0, r1, s1, bv[b][n].x, bv[b][n].y);
-                    mma16816(d, r2, s2, r3, s3, bv[b][n].z, bv[b][n].w);
+                    float (&d0)[4] = FMT == MOE_MXFP4 ? sacc[b][n] : acc[b][n];
+                    float (&d1)[4] = FMT == MOE_MXFP4 ? sacc[NB + b][n] : acc[NB + b][n];
+                    mma16816(d0, p0, t0, p1, t1, bv[b][n].x, bv[b][n].y);
+                    mma16816(d1, p2, t2, p3, t3, bv[b][n].z, bv[b][n].w);
                 }
         }
-    }
-    if (FMT == MOE_MXFP4) {
+        if (FMT == MOE_MXFP4) {
 #pragma unroll
-        for (int t = 0; t < TT; t++)
+            for (int a = 0; a < NA; a++)
 #pragma unroll
-            for (int n = 0; n < NT; n++) {
-                acc[t][n][0] = fmaf(sacc[t][n][0], post[t], acc[t][n][0]);
-                acc[t][n][1] = fmaf(sacc[t][n][1], post[t], acc[t][n][1]);
-                acc[t][n][2] = fmaf(sacc[t][n][2], post8[t], acc[t][n][2]);
-                acc[t][n][3] = fmaf(sacc[t][n][3], post8[t], acc[t][n][3]);
-            }
+                for (int n = 0; n < NT; n++) {
+                    acc[a][n][0] = fmaf(sacc[a][n][0], post, acc[a][n][0]);
+                    acc[a][n][1] = fmaf(sacc[a][n][1], post, acc[a][n][1]);
+                    acc[a][n][2] = fmaf(sacc[a][n][2], post8, acc[a][n][2]);
+                    acc[a][n][3] = fmaf(sacc[a][n][3], post8, acc[a][n][3]);
+                }
+        }
+        c = c_n;
+        c8 = c8_n;
+        u = u_n;
+        u8 = u8_n;
+        code = cn;
+        scl = sn;
     }
+#pragma unroll
+    for (int n = 0; n < NT; n++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            float v = acc[0][n][e];
+#pragma unroll
+            for (int i = 1; i < NA; i++) v += acc[i][n][e];
+            out[n][e] = v;
+        }
 }
 
 // Index (16-byte pieces) of the B-operand piece holding elements k0 .. k0+7
@@ -365,27 +380,10 @@ __device__ __forceinline__ int piece_index(int k0, int n, int N) {
     return ((s * 4 + j) * N + n) * 4 + q;
 }
 
-// Shared-memory byte offset of 16-byte chunk c (0..7) of row r in a box of 128-byte
-// rows written with the 128-byte swizzle (the chunk index XOR the row's low 3 bits).
-__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
-
-// Row of a 16-row tile in shared memory that feeds MMA row i (0..15): rows 2p and
-// 2p+1 of the MMA are read in the same shared-memory phase, so they go to rows p
-// and p + 4, whose swizzled chunks sit in opposite halves of the banks.
-__device__ __forceinline__ int tile_row(int i) { return (i & 8) | ((i & 1) << 2) | ((i & 7) >> 1); }
-
-// Element e (0..3) of lane `lane`'s accumulator holding (row rr, column m) of a
-// 16 x (8 NT) tile: rows g and g+8, columns 2q and 2q+1.
-__device__ __forceinline__ int frag_slot(int rr, int m, int& lane) {
-    const int ml = m & 7;
-    lane = (rr & 7) * 4 + (ml >> 1);
-    return (rr >> 3) * 2 + (ml & 1);
-}
-
 // ------------------------------------------------------------------ the kernel
 
 template <int FMT, int NT>
-__global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant__ FfnArgs a) {
+__global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + a.nstage;
@@ -395,15 +393,12 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant
     float* hinv = xinv + kMaxDecodeT;                                  // [16] per member
     float* hsc = hinv + kMaxDecodeT;                                   // [16] per member
     int* s_misc = reinterpret_cast<int*>(hsc + kMaxDecodeT);           // [8]
-    float* red = reinterpret_cast<float*>(smem + a.o_red);             // [2][kNC][2][NT][32][4]
+    float* pairbuf = reinterpret_cast<float*>(smem + a.o_red);         // [unit][2][2 (gate, up)][ks][16][T]
     float* hloc = reinterpret_cast<float*>(smem + a.o_hloc);           // [2][T][I/C], then [2][T] maxima
     uint4* xf = reinterpret_cast<uint4*>(smem + a.o_x);                // x fragments, N = T
     uint4* hf_hi = reinterpret_cast<uint4*>(smem + a.o_h);             // h fragments, N = T
     uint4* hf_lo = hf_hi + (size_t)a.T * a.I / 8;
-    // the 128-byte swizzle of the TMA boxes follows shared-memory address bits 7..9:
-    // the stage ring starts on a 1024-byte boundary (the launch adds 1 KB of slack)
     uint8_t* stages = smem + a.o_stage;
-    stages += (1024u - (smem_addr(stages) & 1023u)) & 1023u;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     volatile unsigned int* abort_flag = a.ctr + kAbortIdx;
@@ -564,21 +559,15 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant
         trace[14] = (unsigned long long)rho;
     }
 
-    // Stage layouts.  A: gate codes [H/256 boxes][RA rows][128 B], then up codes the
-    // same, then the RA scale rows of gate and of up; B: down codes [I/256 boxes]
-    // [RB rows][128 B], then the RB scale rows.  Boxes are 1024-byte aligned.
+    // Stage layouts (row-major, as in the slot): A = RA code rows of gate, RA of up,
+    // then their RA scale rows each; B = RB code rows of down, then their scale rows.
     const int RA = a.RA, RB = a.RB;
-    const uint32_t boxA = (uint32_t)RA * 128, boxB = (uint32_t)RB * 128;
-    const int nboxA = H / 256, nboxB = I / 256;
-    const uint32_t codesA = (uint32_t)nboxA * boxA;          // one tensor's codes in an A stage
+    const uint32_t CA = (uint32_t)RA * (H / 2);               // one tensor's code bytes in an A stage
+    const uint32_t CB = (uint32_t)RB * (I / 2);
     if (warp == kNC) {
         // ---------------------------------------------------------------- producer
-        const uint32_t txA = 2u * RA * (uint32_t)(H / 2) + 2u * RA * SA;
-        const uint32_t txB = (uint32_t)RB * (uint32_t)(I / 2) + (uint32_t)RB * SB;
-        if (lane == 0) {
-            prefetch_tmap(&a.map_a);
-            prefetch_tmap(&a.map_b);
-        }
+        const uint32_t txA = 2u * CA + 2u * RA * SA;
+        const uint32_t txB = CB + (uint32_t)RB * SB;
         int st = 0;
         uint32_t round = 0;
         int issued = 0;
@@ -593,12 +582,11 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant
                     *abort_flag = 1;
                 }
             }
-            // every lane acquires the ticket itself, then orders its TMA (async
+            // every lane acquires the ticket itself, then orders its bulk (async
             // proxy) reads of the slot after that acquire
             (void)ld_acquire_sys_u32(a.ready + G.slot);
             fence_proxy_async_global();
             const uint8_t* blk = a.slots + (unsigned long long)G.slot * a.block_bytes;
-            const int ya = G.slot * a.rows_a, yb = G.slot * a.rows_b;
             for (int s = 0; s < nA + nB; s++) {
                 bool ok = true;
                 if (lane == 0) ok = mbar_wait_abort(&empty[st], (round & 1) ^ 1, a.pipe_ns, abort_flag);
@@ -611,21 +599,15 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant
                 if (lane == 0) mbar_arrive_expect_tx(&full[st], s < nA ? txA : txB);
                 __syncwarp();
                 if (s < nA) {
-                    const int r0 = rho * IC + RA * s;
-                    for (int bx = lane; bx < 2 * nboxA; bx += 32) {       // gate boxes, then up boxes
-                        const int t = bx >= nboxA, b = bx - t * nboxA;
-                        tma_load_2d(dst + t * codesA + b * boxA, &a.map_a, b * 128,
-                                    ya + (t ? a.row_up : a.row_gate) + r0, &full[st]);
-                    }
-                    if (lane == 0) bulk_g2s(dst + 2 * codesA, blk + a.off[1] + (unsigned long long)r0 * SA, RA * SA, &full[st]);
-                    if (lane == 1)
-                        bulk_g2s(dst + 2 * codesA + RA * SA, blk + a.off[3] + (unsigned long long)r0 * SA, RA * SA, &full[st]);
+                    const unsigned long long r0 = (unsigned long long)(rho * IC + RA * s);
+                    if (lane == 0) bulk_g2s(dst, blk + a.off[0] + r0 * (H / 2), CA, &full[st]);
+                    if (lane == 1) bulk_g2s(dst + CA, blk + a.off[2] + r0 * (H / 2), CA, &full[st]);
+                    if (lane == 2) bulk_g2s(dst + 2 * CA, blk + a.off[1] + r0 * SA, RA * SA, &full[st]);
+                    if (lane == 3) bulk_g2s(dst + 2 * CA + RA * SA, blk + a.off[3] + r0 * SA, RA * SA, &full[st]);
                 } else {
-                    const int r0 = rho * HC + (s - nA) * RB;
-                    for (int b = lane; b < nboxB; b += 32)
-                        tma_load_2d(dst + b * boxB, &a.map_b, b * 128, yb + a.row_down + r0, &full[st]);
-                    if (lane == 0)
-                        bulk_g2s(dst + nboxB * boxB, blk + a.off[5] + (unsigned long long)r0 * SB, RB * SB, &full[st]);
+                    const unsigned long long r0 = (unsigned long long)(rho * HC + (s - nA) * RB);
+                    if (lane == 0) bulk_g2s(dst, blk + a.off[4] + r0 * (I / 2), CB, &full[st]);
+                    if (lane == 1) bulk_g2s(dst + CB, blk + a.off[5] + r0 * SB, RB * SB, &full[st]);
                 }
                 if (trace && lane == 0 && issued < 8) trace[24 + issued] = globaltimer();
                 issued++;
@@ -644,40 +626,36 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant
                     atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
     } else {
         // ---------------------------------------------------------------- consumers
+        // A stage = 16 rows of gate and the same 16 rows of up.  Unit u = warp /
+        // (2 ks) takes A stages u, u + nAU, ...: its even warps the gate tile, its
+        // odd ones the up tile, each over 1/ks of K (part kp = (warp % 2ks) / 2);
+        // the unit then sums the parts in order and forms h.
+        // B stage = RB rows of down, TRB = RB / 16 tiles: warp group warp / TRB takes
+        // B stages group, group + nBU, ..., one tile over the whole K per warp.
+        // nAU and nBU divide the ring size, so within a phase every slot is filled
+        // and emptied for one unit (or group) only, in order: a wait never meets a
+        // slot whose earlier fill is still pending (whose phase parity would
+        // alias).  Consumer barriers separate the phases.
         const int g8 = lane >> 2, q = lane & 3;
-        const int pr = tile_row(g8);                       // shared-memory row of MMA row g8 (g8 + 8: pr + 8)
-        // A: tile pairs (gate tile, up tile) of the stage; warps per pair split K
-        const int TA = RA / 16, WPA = kNC / TA, tpa = warp / WPA, kpa = warp % WPA;
-        // B: RB/16 tiles; warps per tile split K
-        const int TRB = RB / 16, wpt = kNC / TRB, tile = warp % TRB, kpart = warp / TRB;
-        constexpr int kRedStage = kNC * 2 * NT * 32 * 4;   // floats of one red buffer
+        const int ks = a.ks, uw = 2 * ks, unit = warp / uw, widx = warp - unit * uw;
+        const int role = widx & 1, kp = widx >> 1, segsA = nsegA / ks;
+        const int TRB = RB / 16, grp = warp / TRB, tile = warp % TRB;
+        const int nAU = a.nAU, nBU = a.nBU;
+        const uint32_t qs = FMT == MOE_NVFP4 ? 2 * q : 0;   // the thread's scale bytes in a row's segment
         const int bstride = 4 * T;                         // pieces between the words j of a segment
-        int st = 0, rb = 0, it = 0;
-        uint32_t round = 0;
-        auto next_stage = [&]() {
-            rb ^= 1;
-            if (++st == a.nstage) {
-                st = 0;
-                round++;
-            }
-        };
-        auto wait_full = [&]() {
-            if (!mbar_wait_abort(&full[st], round & 1, a.pipe_ns, abort_flag)) {
+        int gi = 0, it = 0, pst = 0;                       // global stage index, group count, pair stages
+        auto slot_wait = [&](int k) {
+            if (!mbar_wait_abort(&full[k % a.nstage], (uint32_t)(k / a.nstage) & 1, a.pipe_ns, abort_flag)) {
                 if (lane == 0) atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
                 *abort_flag = 1;
             }
         };
-        // (MMA row rr, member m) of tile slot t summed over the warps w0, w0 + dw, ...
-        auto red_sum = [&](int t, int rr, int m, int w0, int dw, int nw) {
-            int lx;
-            const int e = frag_slot(rr, m, lx);
-            const int nt = m >> 3;
-            float s = 0.0f;
-            for (int i = 0; i < nw; i++) {
-                const int w = w0 + i * dw;
-                s += red[(size_t)rb * kRedStage + ((((size_t)w * 2 + t) * NT + nt) * 32 + lx) * 4 + e];
-            }
-            return s;
+        // the empty barrier counts kNC arrivals per stage: each of the n warps of a stage gives kNC / n
+        auto slot_release = [&](int k, int n) {
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;"
+                             ::"r"(smem_addr(&empty[k % a.nstage])), "r"(kNC / n) : "memory");
         };
         for (int g = cid; g < ng; g += ncl, it++) {
             const Group& G = groups[g];
@@ -685,65 +663,59 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant
             float* hl = hloc + (size_t)hb * T * IC;                        // [M][IC] this CTA's slice of h
             unsigned* hmx = reinterpret_cast<unsigned*>(hloc + (size_t)2 * T * IC) + hb * T;   // [M] |h| max
             if (tid < T) hmx[tid] = 0u;
+            named_sync(1, kConsThreads);     // hmx is zero before any pair adds to it
             // this lane's B columns: member m = g8 + 8 nt of the group (null past M)
-            const uint4* xcol[NT];
-            const uint4* hcol_hi[NT];
-            const uint4* hcol_lo[NT];
+            const uint4* xb[1][NT];            // x of the member's token
+            const uint4* hb2[2][NT];           // h of the member: high parts, remainders
 #pragma unroll
             for (int nt = 0; nt < NT; nt++) {
                 const int m = g8 + 8 * nt;
-                xcol[nt] = m < M ? xf + (size_t)G.tok[m] * 4 + q : nullptr;
-                hcol_hi[nt] = m < M ? hf_hi + (size_t)m * 4 + q : nullptr;
-                hcol_lo[nt] = m < M ? hf_lo + (size_t)m * 4 + q : nullptr;
+                xb[0][nt] = m < M ? xf + (size_t)G.tok[m] * 4 + q : nullptr;
+                hb2[0][nt] = m < M ? hf_hi + (size_t)m * 4 + q : nullptr;
+                hb2[1][nt] = m < M ? hf_lo + (size_t)m * 4 + q : nullptr;
             }
 
-            // ---- A: RA rows of gate and the same RA rows of up per stage
+            // ---- A: stage s = gate rows [rho*IC + 16 s, +16) and the same rows of up
             for (int s = 0; s < nA; s++) {
-                wait_full();
+                const int k = gi + s;
+                if (unit >= nAU || s % nAU != unit) continue;
+                slot_wait(k);
                 if (trace && tid == 0 && it == 0 && s == 0) trace[4] = globaltimer();
-                if (trace && tid == 0 && it == 0 && s < 8) trace[16 + s] = globaltimer();
-                const uint8_t* sb = stages + (size_t)st * a.stage_bytes;
-                float acc[2][NT][4];
+                if (trace && lane == 0 && widx == 0 && it == 0 && s < 8) trace[16 + s] = globaltimer();
+                const uint8_t* sb = stages + (size_t)(k % a.nstage) * a.stage_bytes;
+                const uint8_t* tb = sb + role * CA;                       // gate or up codes
+                const uint8_t* tsc = sb + 2 * CA + role * RA * SA;        // their scale rows
+                float part[NT][4];
+                tile_mma<FMT, NT, 1>(tb + g8 * (H / 2) + 16 * q, 8 * (H / 2), tsc + g8 * SA + qs, 8 * SA, q,
+                                     kp * segsA, segsA, xb, bstride, part);
+                slot_release(k, uw);
+                // the unit's parts: [parity][role][kp][16][T]
+                float* ub = pairbuf + (size_t)unit * 2 * 2 * ks * 16 * T + (size_t)(pst & 1) * 2 * ks * 16 * T;
+                float* pb = ub + (size_t)(role * ks + kp) * 16 * T;
 #pragma unroll
-                for (int t = 0; t < 2; t++)
+                for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-                    for (int nt = 0; nt < NT; nt++)
-#pragma unroll
-                        for (int e = 0; e < 4; e++) acc[t][nt][e] = 0.0f;
-                const int row = tpa * 16 + pr;                   // shared-memory row of MMA row g8
-                for (int seg = kpa; seg < nsegA; seg += WPA) {
-                    const uint32_t so = FMT == MOE_NVFP4 ? seg * 8 + 2 * q : seg * 4;
-                    const uint32_t co = (seg >> 1) * boxA + swz(row, ((seg & 1) << 2) | q);
-                    const uint8_t* code[2] = {sb + co, sb + codesA + co};
-                    const uint8_t* scl[2] = {sb + 2 * codesA + row * SA + so, sb + 2 * codesA + (RA + row) * SA + so};
-                    const uint4* bp[1][NT];
-#pragma unroll
-                    for (int nt = 0; nt < NT; nt++)
-                        bp[0][nt] = xcol[nt] ? xcol[nt] + (size_t)seg * 4 * bstride : nullptr;
-                    seg_mma<FMT, 2, NT, 1>(code, 8 * 128, scl, 8 * SA, q, bp, bstride, acc);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[st]);
-                float4* rp = reinterpret_cast<float4*>(red + (size_t)rb * kRedStage);
-#pragma unroll
-                for (int t = 0; t < 2; t++)
-#pragma unroll
-                    for (int nt = 0; nt < NT; nt++)
-                        rp[(((size_t)warp * 2 + t) * NT + nt) * 32 + lane] =
-                            make_float4(acc[t][nt][0], acc[t][nt][1], acc[t][nt][2], acc[t][nt][3]);
-                named_sync(1, kConsThreads);
-                for (int o = tid; o < RA * M; o += kConsThreads) {
-                    const int pair = o / (16 * M), rem = o - pair * 16 * M, rr = rem & 15, m = rem >> 4;
-                    const int w0 = pair * WPA;
-                    const float gs = red_sum(0, rr, m, w0, 1, WPA), us = red_sum(1, rr, m, w0, 1, WPA);
-                    const float xs = xinv[G.tok[m]] * 16384.0f;     // undo x's scale and the decode's 2^-14
+                    for (int e = 0; e < 4; e++) {
+                        const int rr = g8 + (e >> 1) * 8, m = 8 * nt + 2 * q + (e & 1);
+                        if (m < M) pb[rr * T + m] = part[nt][e];
+                    }
+                named_sync(2 + unit, 32 * uw);
+                for (int o = widx * 32 + lane; o < 16 * M; o += 32 * uw) {
+                    const int rr = o & 15, m = o >> 4;
+                    float gs = ub[rr * T + m], us = ub[(size_t)ks * 16 * T + rr * T + m];
+                    for (int p = 1; p < ks; p++) {
+                        gs += ub[(size_t)p * 16 * T + rr * T + m];
+                        us += ub[(size_t)(ks + p) * 16 * T + rr * T + m];
+                    }
+                    const float xs = xinv[G.tok[m]];                   // undo x's scale
                     const float gv = gs * xs * G.ts[0], uv = us * xs * G.ts[1];
                     const float hv = gv / (1.0f + expf(-gv)) * uv;
-                    hl[m * IC + s * RA + pair * 16 + tile_row(rr)] = hv;
+                    hl[m * IC + s * 16 + rr] = hv;
                     atomicMax(hmx + m, __float_as_uint(fabsf(hv)));
                 }
-                next_stage();
+                pst++;
             }
+            gi += nA;
             named_sync(1, kConsThreads);     // every row of this CTA's slice of h is written
             if (trace && tid == 0 && it == 0) trace[5] = globaltimer();
 
@@ -787,47 +759,30 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant
             named_sync(1, kConsThreads);
             if (trace && tid == 0 && it == 0) trace[7] = globaltimer();
 
-            // ---- B: RB rows of down per stage; warps on tile (warp % TRB), K part warp / TRB
-            for (int s = 0; s < nB; s++) {
-                wait_full();
-                if (trace && tid == 0 && it == 0 && nA + s < 8) trace[16 + nA + s] = globaltimer();
-                const uint8_t* sb = stages + (size_t)st * a.stage_bytes;
-                float acc[1][NT][4];
+            // ---- B: stage b = down rows [rho*HC + RB b, +RB); warp `tile` of group b % ngrp
+            for (int b = 0; b < nB; b++) {
+                const int k = gi + b;
+                if (b % nBU != grp) continue;
+                slot_wait(k);
+                if (trace && lane == 0 && tile == 0 && it == 0 && nA + b < 8) trace[16 + nA + b] = globaltimer();
+                const uint8_t* sb = stages + (size_t)(k % a.nstage) * a.stage_bytes;
+                const int row = tile * 16 + g8;
+                float acc[NT][4];
+                tile_mma<FMT, NT, 2>(sb + row * (I / 2) + 16 * q, 8 * (I / 2), sb + CB + row * SB + qs, 8 * SB, q,
+                                     0, nsegB, hb2, bstride, acc);
+                slot_release(k, TRB);
+                const int r0 = rho * HC + b * RB + tile * 16;
 #pragma unroll
                 for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-                    for (int e = 0; e < 4; e++) acc[0][nt][e] = 0.0f;
-                const int row = tile * 16 + pr;
-                for (int seg = kpart; seg < nsegB; seg += wpt) {
-                    const uint32_t so = FMT == MOE_NVFP4 ? seg * 8 + 2 * q : seg * 4;
-                    const uint8_t* code[1] = {sb + (seg >> 1) * boxB + swz(row, ((seg & 1) << 2) | q)};
-                    const uint8_t* scl[1] = {sb + nboxB * boxB + row * SB + so};
-                    const uint4* bp[2][NT];
-#pragma unroll
-                    for (int nt = 0; nt < NT; nt++) {
-                        bp[0][nt] = hcol_hi[nt] ? hcol_hi[nt] + (size_t)seg * 4 * bstride : nullptr;
-                        bp[1][nt] = hcol_lo[nt] ? hcol_lo[nt] + (size_t)seg * 4 * bstride : nullptr;
+                    for (int e = 0; e < 4; e++) {
+                        const int rr = g8 + (e >> 1) * 8, m = 8 * nt + 2 * q + (e & 1);
+                        if (m < M)
+                            a.y_part[((size_t)G.tok[m] * a.k + G.rank[m]) * H + r0 + rr] =
+                                G.wt[m] * (acc[nt][e] * hinv[m] * G.ts[2]);
                     }
-                    seg_mma<FMT, 1, NT, 2>(code, 8 * 128, scl, 8 * SB, q, bp, bstride, acc);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[st]);
-                float4* rp = reinterpret_cast<float4*>(red + (size_t)rb * kRedStage);
-#pragma unroll
-                for (int nt = 0; nt < NT; nt++)
-                    rp[(((size_t)warp * 2) * NT + nt) * 32 + lane] =
-                        make_float4(acc[0][nt][0], acc[0][nt][1], acc[0][nt][2], acc[0][nt][3]);
-                named_sync(1, kConsThreads);
-                const int r0 = rho * HC + s * RB;
-                for (int o = tid; o < TRB * 16 * M; o += kConsThreads) {
-                    const int tl = o / (16 * M), rem = o - tl * 16 * M, rr = rem & 15, m = rem >> 4;
-                    const float ys = red_sum(0, rr, m, tl, TRB, wpt);
-                    const int yrow = r0 + tl * 16 + tile_row(rr);
-                    a.y_part[((size_t)G.tok[m] * a.k + G.rank[m]) * H + yrow] =
-                        G.wt[m] * (ys * (hinv[m] * 16384.0f) * G.ts[2]);
-                }
-                next_stage();
             }
+            gi += nB;
 
             // ---- this group's rows of block rho are in y_part: count it; the last
             // group to finish the block sums it over the ranks (K5)
@@ -841,18 +796,19 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const __grid_constant
             }
             named_sync(1, kConsThreads);
             if (s_misc[1]) {
-                if (a.y) {
-                    const int q4 = HC / 4;
-                    for (int v = tid; v < T * q4; v += kConsThreads) {
-                        const int t = v / q4, r = rho * HC + (v - t * q4) * 4;
-                        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                        for (int j = 0; j < a.k; j++) {
-                            const float4 pv = __ldcg(reinterpret_cast<const float4*>(a.y_part + ((size_t)t * a.k + j) * H + r));
-                            sum.x += pv.x;
-                            sum.y += pv.y;
-                            sum.z += pv.z;
-                            sum.w += pv.w;
-                        }
+                // y = the rank-ordered sum of y_part, rounded to bf16
+                const int q4 = HC / 4;
+                for (int v = tid; v < T * q4; v += kConsThreads) {
+                    const int t = v / q4, r = rho * HC + (v - t * q4) * 4;
+                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int j = 0; j < a.k; j++) {
+                        const float4 pv = __ldcg(reinterpret_cast<const float4*>(a.y_part + ((size_t)t * a.k + j) * H + r));
+                        sum.x += pv.x;
+                        sum.y += pv.y;
+                        sum.z += pv.z;
+                        sum.w += pv.w;
+                    }
+                    if (a.y) {
                         const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(sum.x));
                         const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(sum.y));
                         const uint32_t b2 = __bfloat16_as_ushort(__float2bfloat16_rn(sum.z));
@@ -938,21 +894,19 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
 
 static size_t up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
-int make_tmap_2d(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint64_t pitch,
-                 uint32_t box_bytes, uint32_t box_rows, bool swizzle128);
-
-// Shared-memory layout and stage sizes of one launch: RA = 32 gate rows per A
-// stage when two such stages fit, else 16; RB = the most down rows (128, 64, 32
-// or 16, dividing H/C) whose stage is no larger than an A stage.  MOE_EINVAL if
-// not even two stages fit.
+// Shared-memory layout and stage sizes of one launch.  A CTA streams at HBM rate
+// only with several stages in flight, so stages are small: RA = 16 gate (and up)
+// rows per A stage (one 16-row tile of each); RB = the most down rows
+// (128, 64, 32 or 16, dividing H/C) whose stage is no larger than an A stage.
+// MOE_EINVAL if not even two stages fit.
 static int plan_ffn(const moe_pool* p, int T, int C, int NT, FfnArgs& a, size_t& smem) {
     const moe_config& c = p->cfg;
     const int bs = p->bs;
     const int IC = c.I / C, HC = c.H / C;
     const size_t SA = c.H / bs, SB = c.I / bs;
     const size_t budget = (size_t)p->ffn_smem;
-    for (int RA = 32; RA >= 16; RA >>= 1) {
-        if (IC % RA) continue;
+    {
+        const int RA = 16;
         const size_t stA = 2 * (size_t)RA * (c.H / 2) + 2 * (size_t)RA * SA;
         int RB = 16;
         for (int rb = 128; rb >= 16; rb >>= 1)
@@ -963,61 +917,53 @@ static int plan_ffn(const moe_pool* p, int T, int C, int NT, FfnArgs& a, size_t&
         a.RA = RA;
         a.RB = RB;
         const size_t stB = (size_t)RB * (c.I / 2 + SB);
-        a.stage_bytes = (int)up(std::max(stA, stB), 1024);
+        a.stage_bytes = (int)up(std::max(stA, stB), 128);
         size_t o = up((2 * 16 + 2) * sizeof(uint64_t), 128);
         a.o_groups = (int)o;
         o += sizeof(Group) * kMaxDecodePairs;
         a.o_misc = (int)up(o, 16);
         o = a.o_misc + 3 * kMaxDecodeT * sizeof(float) + 8 * sizeof(int);
         a.o_red = (int)up(o, 16);
-        o = a.o_red + (size_t)2 * kNC * 2 * NT * 32 * 4 * sizeof(float);
+        o = a.o_red + (size_t)(kNC / 2) * 2 * 2 * 16 * T * sizeof(float);   // units * ks <= 4
         a.o_hloc = (int)up(o, 16);
         o = a.o_hloc + ((size_t)2 * T * IC + 2 * T) * sizeof(float);
         a.o_x = (int)up(o, 16);
         o = a.o_x + (size_t)T * c.H * 2;
         a.o_h = (int)up(o, 16);
         o = a.o_h + (size_t)2 * T * c.I * 2;
-        a.o_stage = (int)up(o, 1024);
+        a.o_stage = (int)up(o, 128);
         // the prologue keeps its per-(token, rank) table (7 ints + 3 floats each) in the ring
         const size_t need_ring = std::max((size_t)2 * a.stage_bytes, (size_t)10 * 4 * kMaxDecodePairs);
-        if (a.o_stage + need_ring + 1024 > budget) continue;
-        a.nstage = (int)std::min<size_t>(8, (budget - a.o_stage - 1024) / a.stage_bytes);
-        smem = a.o_stage + (size_t)a.nstage * a.stage_bytes + 1024;
+        if (a.o_stage + need_ring > budget)
+            return fail(MOE_EINVAL, "decode FFN: T * (H + 2 I) too large for shared memory (lower max_tokens)");
+        a.nstage = (int)std::min<size_t>(8, (budget - a.o_stage) / a.stage_bytes);
+        if (a.nstage >= kNC / 2) a.nstage = a.nstage / (kNC / 2) * (kNC / 2);
+        smem = a.o_stage + (size_t)a.nstage * a.stage_bytes;
+        // A: units of 2 ks warps, as many as divide the ring; the K split with the
+        // fewest rounds (one round = one stage's full-K dot products / ks) wins,
+        // a little weight against more warps meeting at every stage
+        const int nA = IC / RA, nsegA = c.H / 128;
+        double best = 1e30;
+        for (int ks = 1; ks <= kNC / 2; ks *= 2) {
+            if (nsegA % ks) continue;
+            int u = std::min(kNC / (2 * ks), a.nstage);
+            while (a.nstage % u) u--;
+            const double cost = (double)((nA + u - 1) / u) / ks + 0.05 * ks;
+            if (cost < best) {
+                best = cost;
+                a.ks = ks;
+                a.nAU = u;
+            }
+        }
+        // B: groups of RB / 16 warps, as many as divide the ring
+        a.nBU = 1;
+        for (int d = kNC / (a.RB / 16); d >= 1; d--)
+            if (a.nstage % d == 0) {
+                a.nBU = d;
+                break;
+            }
         return MOE_OK;
     }
-    return fail(MOE_EINVAL, "decode FFN: T * (H + 2 I) too large for shared memory (lower max_tokens)");
-}
-
-// The 2-D views of the pool's code rows (boxes 128 bytes x `rows`), built once
-// per pool and box height.  The FP4 code rows of every slot must sit at whole
-// rows of the view: block bytes and tensor offsets multiples of the row bytes.
-static int ffn_maps(moe_pool* p, FfnArgs& a) {
-    const moe_config& c = p->cfg;
-    const uint64_t rwa = c.H / 2, rwb = c.I / 2, blk = p->lay.bytes;
-    if (blk % rwa || p->lay.off[0] % rwa || p->lay.off[2] % rwa || blk % rwb || p->lay.off[4] % rwb)
-        return fail(MOE_EINVAL, "decode FFN: the expert block does not divide into rows of H/2 and I/2 bytes");
-    const uint64_t pool_bytes = (uint64_t)c.n_slots * blk;
-    if (pool_bytes / rwa > 0x7fffffffull) return fail(MOE_EINVAL, "decode FFN: slot pool too large for a 2-D view");
-    const int ia = a.RA == 32 ? 1 : 0;
-    int ib = 0;
-    while ((16 << ib) < a.RB) ib++;
-    int rc;
-    if (!p->ffn_map_a_ok[ia]) {
-        if ((rc = make_tmap_2d(&p->ffn_map_a[ia], p->slots, rwa, pool_bytes / rwa, rwa, 128, a.RA, true))) return rc;
-        p->ffn_map_a_ok[ia] = 1;
-    }
-    if (!p->ffn_map_b_ok[ib]) {
-        if ((rc = make_tmap_2d(&p->ffn_map_b[ib], p->slots, rwb, pool_bytes / rwb, rwb, 128, a.RB, true))) return rc;
-        p->ffn_map_b_ok[ib] = 1;
-    }
-    a.map_a = p->ffn_map_a[ia];
-    a.map_b = p->ffn_map_b[ib];
-    a.rows_a = (int)(blk / rwa);
-    a.rows_b = (int)(blk / rwb);
-    a.row_gate = (int)(p->lay.off[0] / rwa);
-    a.row_up = (int)(p->lay.off[2] / rwa);
-    a.row_down = (int)(p->lay.off[4] / rwb);
-    return MOE_OK;
 }
 
 // For every cluster size C in {16, 8, 4, 2, 1} that splits I and H into 16-row
@@ -1073,28 +1019,28 @@ static int query_clusters(moe_pool* p, int (&ncl)[5]) {
 // the smallest, then the fewest rounds, then the larger C.
 static int g_force_cluster = 0;   // moe_set_ffn_cluster: 0 = automatic
 
-static void choose_cluster(const int (&ncl)[5], int groups, int& C, int& nclusters) {
-    if (g_force_cluster > 0)
-        for (int ci = 0, c = kMaxCluster; ci < 5; ci++, c >>= 1)
-            if (c == g_force_cluster && ncl[ci] > 0) {
-                C = c;
-                nclusters = std::min(ncl[ci], groups);
-                return;
-            }
+// Cluster size C of a launch: the work of one expert is split over C CTAs, and
+// the clusters that fit at once take the G unique experts in ceil(G / clusters)
+// rounds, so the time goes as rounds * (1 / C + the fixed cost of a group, about
+// 4 % of an expert on one CTA).  G is the expected number of unique experts,
+// E (1 - (1 - k/E)^T) (at most T * k).
+static void choose_cluster(const moe_pool* p, const int (&ncl)[5], int T, int& C, int& nclusters) {
+    const moe_config& c = p->cfg;
+    const double Gd = c.E * (1.0 - std::pow(1.0 - (double)c.k / c.E, (double)T));
+    const int G = std::max(1, std::min(T * c.k, (int)(Gd + 0.5)));
     double best = 1e30;
-    int best_rounds = 1 << 30;
     C = 1;
     nclusters = 1;
-    for (int ci = 0, c = kMaxCluster; ci < 5; ci++, c >>= 1) {
+    for (int ci = 0, cc = kMaxCluster; ci < 5; ci++, cc >>= 1) {
         if (ncl[ci] <= 0) continue;
-        const int n = std::min(ncl[ci], groups);
-        const int rounds = (groups + n - 1) / n;
-        const double cost = (double)rounds / c;
-        if (cost < best - 1e-12 || (cost < best + 1e-12 && rounds < best_rounds)) {
+        if (g_force_cluster && cc != g_force_cluster) continue;
+        const int n = std::min(ncl[ci], G);
+        const int rounds = (G + n - 1) / n;
+        const double cost = rounds * (1.0 / cc + 0.04);
+        if (cost < best - 1e-12) {
             best = cost;
-            best_rounds = rounds;
-            C = c;
-            nclusters = n;
+            C = cc;
+            nclusters = std::min(ncl[ci], T * c.k);
         }
     }
 }
@@ -1107,11 +1053,8 @@ static int ffn_shape(moe_pool* p, FfnArgs& a, size_t& smem, int& nclusters) {
         if (rc) return rc;
         p->ffn_attr_set[fi][ni] = 1;
     }
-    // a call has at most T * k unique experts, one cluster each
-    choose_cluster(p->ffn_ncl[fi][ni], a.T * a.k, a.C, nclusters);
-    int rc = plan_ffn(p, a.T, a.C, NT, a, smem);
-    if (rc) return rc;
-    return ffn_maps(p, a);
+    choose_cluster(p, p->ffn_ncl[fi][ni], a.T, a.C, nclusters);
+    return plan_ffn(p, a.T, a.C, NT, a, smem);
 }
 
 template <int FMT, int NT>
@@ -1205,8 +1148,6 @@ extern "C" int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_m
 extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx,
                               const float* w, const int32_t* slot_of, float* y_part, void* y_bf16, int* status,
                               void* stream) {
-    static_assert(offsetof(FfnArgs, map_a) % 64 == 0 && offsetof(FfnArgs, map_b) % 64 == 0,
-                  "tensor maps must be 64-byte aligned in the kernel parameters");
     if (!p || !x_bf16 || !idx || !w || !slot_of || !y_part || !status) return fail(MOE_EINVAL, "null argument");
     const moe_config& c = p->cfg;
     if (layer < 0 || layer >= c.L) return fail(MOE_EBOUNDS, "layer outside the pool");

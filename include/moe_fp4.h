@@ -279,10 +279,10 @@ int moe_expert_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const i
  * Process-wide; affects later launches.  Errors: MOE_EINVAL (non-positive). */
 int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
 
-/* Cluster size of later moe_expert_ffn launches (for tuning sweeps): 1, 2, 4,
- * 8 or 16 CTAs per expert where the shapes and the GPU allow it (otherwise the
- * automatic choice), 0 = automatic (the default: the size with the least work
- * per CTA counting the rounds in which the clusters take the experts).
+/* Cluster size of later moe_expert_ffn launches (for tuning sweeps): 1, 2, 4, 8
+ * or 16 CTAs per expert where the shapes and the GPU allow it (otherwise the
+ * automatic choice); 0 = automatic (the default: the size with the least work
+ * per CTA, counting the rounds in which the clusters take the experts).
  * Process-wide.  Errors: MOE_EINVAL. */
 int moe_set_ffn_cluster(int cluster);
 
