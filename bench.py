@@ -161,7 +161,8 @@ def make_pool(m, w, n_slots, T, host_layers, experts):
 def preload(torch, m, pool, w):
     """Make every (layer, expert) resident: one lookup of all E experts per layer
     (k distinct per row) and its miss streaming."""
-    idx = torch.arange(w.E, dtype=torch.int32, device="cuda").view(-1, w.k)
+    rows = (w.E + w.k - 1) // w.k         # the last row wraps around to expert 0, 1, ...
+    idx = (torch.arange(rows * w.k, dtype=torch.int32, device="cuda") % w.E).view(rows, w.k)
     slot_of = torch.empty_like(idx)
     cs = torch.cuda.Stream()
     for l in range(w.L):
@@ -335,7 +336,6 @@ def ffn_only(args, w, T):
     import expert_offload_fp4_b200 as m
     pool = make_pool(m, wl, wl.L * wl.E, 8, 1, experts)
     preload(torch, m, pool, wl)
-    m.set_ffn_cluster(args.ffn_cluster)
     xs = np.stack([gen.activations(wl, l, 0, T) for l in range(wl.L)])
     x_dev = torch.from_numpy(xs.view(np.int16)).cuda().view(torch.bfloat16)
     wr = torch.from_numpy(gen.router_weight(wl, 0).view(np.int16)).cuda().view(torch.bfloat16)
@@ -346,17 +346,21 @@ def ffn_only(args, w, T):
     if args.trace:
         buf = torch.zeros((148 * 2, 32), dtype=torch.int64, device="cuda")
         m._lib.load().moe_set_ffn_trace(C_ptr(buf))
-        ffn_roofline(torch, m, wl, pool, T, x_dev, wr, bias, reps=1)
+        ms_traced, _ = ffn_roofline(torch, m, wl, pool, T, x_dev, wr, bias, reps=1)
         m._lib.load().moe_set_ffn_trace(None)
         tr = buf.cpu().numpy()
-        n_cta = info["cluster"] * info["clusters"]
+        n_cta = info["ctas"]
         tr = tr[:n_cta].astype(np.float64)
         t0 = tr[:, 0].min()
-        names = ["start", "staged", "pdl", "table", "first_data", "a_done", "published", "gathered",
-                 "b_done", "counted", "end", "last_copy"]
+        names = {0: "start", 1: "staged", 2: "pdl", 3: "table", 4: "first_data", 5: "a_done",
+                 6: "h_ready", 7: "h_staged", 8: "b_done", 9: "producer_fenced", 10: "end", 11: "last_copy"}
         phases = {nm: [round(float(np.median(tr[:, i] - t0)) / 1e3, 2), round(float((tr[:, i] - t0).max()) / 1e3, 2)]
-                  for i, nm in enumerate(names)}
-        phases["groups_per_cta_max"] = int(tr[:, 12].max())
+                  for i, nm in names.items()}
+        phases["a_items_max"] = int(tr[:, 12].max())
+        phases["b_tiles_max"] = int(tr[:, 13].max())
+        phases["ks"] = sorted(set(int(v) for v in tr[:, 14]))
+        phases["kb"] = sorted(set(int(v) for v in tr[:, 15]))
+        phases["traced_launch_ms"] = round(ms_traced, 5)
         phases["stage_landed"] = [round(float(np.median(tr[:, 16 + i] - t0)) / 1e3, 2) for i in range(8)]
         phases["stage_issued"] = [round(float(np.median(tr[:, 24 + i] - t0)) / 1e3, 2) for i in range(8)]
     pool.close()
@@ -560,8 +564,8 @@ def main():
                     help="ffn: only the decode FFN kernel on a small all-resident pool "
                          "(a few layers), e.g. for an ncu capture")
     ap.add_argument("--layers", type=int, default=4, help="layer positions in --mode ffn")
-    ap.add_argument("--ffn-cluster", type=int, default=0,
-                    help="--mode ffn: force the decode FFN's cluster size (0: automatic)")
+    ap.add_argument("--workload", default="decode_35b", choices=["decode_35b", "decode_284b"],
+                    help="--mode ffn: the layer shapes")
     ap.add_argument("--trace", action="store_true", help="--mode ffn: per-CTA phase stamps")
     ap.add_argument("--host-layers", type=int, default=8,
                     help="--mode offload: distinct host copies of the 40 layers (pinned RAM)")
@@ -597,7 +601,7 @@ def main():
         return
 
     if args.mode == "ffn":
-        return ffn_only(args, w, T)
+        return ffn_only(args, W.DECODE_284B if args.workload == "decode_284b" else w, T)
     if args.mode == "offload":
         return offload_mode(args)
     if args.mode == "prefill":

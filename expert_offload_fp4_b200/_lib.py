@@ -79,7 +79,6 @@ SIGNATURES = {
     "moe_pool_resize": (i32, [vp, i32]),
     "moe_lru_plan_resize": (i32, [vp, vp, i32, i32, vp, C.POINTER(i32), vp, vp, C.POINTER(i32)]),
     "moe_set_ffn_trace": (i32, [vp]),
-    "moe_set_ffn_cluster": (i32, [i32]),
     "moe_ffn_launch_info": (i32, [vp, i32, vp, vp, vp, vp]),
     "moe_expert_ffn": (i32, [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp]),
     "moe_combine": (i32, [vp, i32, i32, i32, vp, vp]),

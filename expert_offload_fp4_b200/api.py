@@ -185,17 +185,12 @@ def expert_ffn(pool, layer, x, idx, w, slot_of, y_part, status, y=None, stream=N
         _s(stream)))
 
 
-def set_ffn_cluster(cluster=0):
-    """moe_set_ffn_cluster: CTAs per expert of later decode FFN launches (0 = automatic)."""
-    L.check("moe_set_ffn_cluster", L.load().moe_set_ffn_cluster(int(cluster)))
-
-
 def ffn_launch_info(pool, T):
     """moe_ffn_launch_info: the decode FFN's launch shape for T tokens on this pool."""
-    c, n, st, sm = C.c_int(), C.c_int(), C.c_int(), C.c_int()
+    c, st, sb, sm = C.c_int(), C.c_int(), C.c_int(), C.c_int()
     L.check("moe_ffn_launch_info", pool.lib.moe_ffn_launch_info(
-        pool.handle, int(T), C.byref(c), C.byref(n), C.byref(st), C.byref(sm)))
-    return dict(cluster=c.value, clusters=n.value, stages=st.value, smem_bytes=sm.value)
+        pool.handle, int(T), C.byref(c), C.byref(st), C.byref(sb), C.byref(sm)))
+    return dict(ctas=c.value, stages=st.value, stage_bytes=sb.value, smem_bytes=sm.value)
 
 
 def decode_layer(pool, layer, x, wr, bias, renormalize, idx, w, slot_of, y_part, y, status, ws,

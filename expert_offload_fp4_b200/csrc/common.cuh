@@ -96,14 +96,15 @@ struct moe_pool {
     int lk_seq;                   // sequence number of the last launched lookup
     int lk_pending;               // a launched lookup whose record was not collected
     int lk_attr_set;
-    // decode FFN counters: [0, 16) groups done per row block (the fused combine),
-    // then the abort flag and the count of finished CTAs
+    // decode FFN counters: [0, H/16) groups done per 16-row tile of H (the fused
+    // combine), then per group the h values published, per (token, rank) the
+    // largest |h| (float bits), kMaxDecodePairs words each, then the abort flag
+    // and the count of finished CTAs
     unsigned int* ctr;
+    float* hbuf;                  // decode FFN: [kMaxDecodePairs][I] h of each (token, rank)
     // copy engine ready-flag write
     void* write_value32;          // cuStreamWriteValue32 entry point
-    int ffn_attr_set[2][2];       // decode FFN launch attributes set, per (format, token tiles)
-    int ffn_ncl[2][2][5];         // clusters of 16, 8, 4, 2, 1 CTAs that fit on the GPU at once
-                                  // (0: that size does not split the pool's shapes)
+    int ffn_grid[2][2];           // decode FFN CTAs per launch (0: not yet set up), per (format, token tiles)
     moe_stats stats;
 };
 

@@ -1,27 +1,29 @@
 // K4 decode expert FFN with the K5 combine fused in, and the slot dequantiser.
 //
-// Work split: one thread-block cluster of C CTAs (C = 16 where the GPU can
-// co-schedule it) per unique expert ("group") of the call; clusters loop over
-// the groups in ticket order (resident experts first, missed ones in the order
-// the copy engine delivers them).  CTA rho of a cluster
-//   A: computes rows [rho*I/C, (rho+1)*I/C) of gate and up for every token of the
-//      group and its slice of h = silu(gate x) * (up x);
-//   X: publishes the slice to the other CTAs of the cluster (an mbarrier arrive
-//      in each peer's shared memory) and gathers the whole h from theirs
-//      (distributed shared memory);
-//   B: computes rows [rho*H/C, (rho+1)*H/C) of y_e = down h, weighted by the
-//      routing weight of each (token, rank), into y_part.
-// Every dependency stays inside the cluster, whose CTAs the hardware runs
-// together, so no CTA ever waits for one that may not be resident.  The last
-// CTA to finish a block of H/C rows (an atomic count over all groups) sums
-// y_part over the ranks in rank order and writes the bf16 output rows (K5).
+// Work split over the whole GPU, one CTA per SM.  The call's unique experts
+// ("groups", in ticket order: resident experts first, missed ones in the order
+// the copy engine delivers them) give two lists of equal-sized work items:
+//   A items: 16 rows of gate and the same 16 rows of up of one group; their dot
+//      products with the x of every member token give 16 rows of
+//      h = silu(gate x) * (up x), stored in fp32 to a global buffer (one row of I
+//      values per (token, rank)) and counted per group;
+//   B tiles: 16 rows of down of one group; once the group's whole h is counted,
+//      y_e = down h for each member, times its routing weight, goes to y_part.
+// CTA c takes the c-th contiguous share of each list (A first, then B), so every
+// SM streams the same number of weight bytes whatever the number of groups.  B
+// waits (bounded) for A items of other CTAs; all CTAs are resident at once (one
+// per SM), and A items wait for nothing but their own copies and tickets, so the
+// waits always end.  The warp that lands the last group of a 16-row tile of H
+// (an atomic count per tile) sums y_part over the ranks in rank order and writes
+// the tile's bf16 output rows (K5).
 //
-// Warp specialisation: warp 8 (the producer) streams the FP4 code rows and
-// block scales of each work stage with 1-D bulk copies (a whole tile of rows is
-// one contiguous range of the slot) into a ring of shared-memory stages
-// (mbarrier full/empty pairs); for a missed expert it first waits (bounded) for
-// the slot's ready ticket written by the copy stream.
-// Warps 0..7 (consumers) run the dot products on the tensor cores with
+// Warp specialisation: warp 16 (the producer) streams the FP4 code rows and
+// block scales of each work stage with 1-D bulk copies (a tile of rows is one
+// contiguous range of the slot) into a ring of shared-memory stages (mbarrier
+// full/empty pairs); for a missed expert it first waits (bounded) for the
+// slot's ready ticket written by the copy stream.  B stages are prefetched
+// while h is still being produced elsewhere.
+// Warps 0..15 (consumers) run the dot products on the tensor cores with
 // mma.sync m16n8k16, f16 inputs and fp32 accumulation:
 //  - weights: E2M1 code pairs converted to f16 pairs (cvt.rn.f16x2.e2m1x2),
 //    multiplied (exactly) by their block scale in f16: the E4M3 scale itself
@@ -30,25 +32,21 @@
 //  - activations: x of each token times a power of two (bf16 is exact in f16
 //    that way); h of each (token, expert) times a power of two and split into
 //    an f16 high part and an f16 remainder, so down h is carried to ~22 bits;
-//  - products are exact, sums fp32; every output row is one warp's chain of
-//    MMAs over the whole K, in a fixed order, so results are reproducible.
+//  - products are exact, sums fp32 in a fixed order, so results are reproducible.
 #include <math.h>
 
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kNC = 8;                       // consumer warps
+constexpr int kNC = 16;                      // consumer warps
 constexpr int kFfnThreads = (kNC + 1) * 32;  // + one producer warp
 constexpr int kConsThreads = kNC * 32;
-// Register cap.  The 9 warps of a CTA spread over the SM's 4 sub-partitions, 3 on
+// Register cap.  The 17 warps of a CTA spread over the SM's 4 sub-partitions, 5 on
 // one of them, whose register file holds 16384 registers; one warp of the SM copy
 // kernel (128 threads, at most 32 registers), which a waiting FFN may depend on,
-// must fit beside them: 3 * 32 * 160 + 32 * 32 <= 16384.
-constexpr int kFfnMaxRegs = 160;
-constexpr int kAbortIdx = kMaxDecodePairs;   // ctr[kAbortIdx] = abort flag
-constexpr int kDoneIdx = kMaxDecodePairs + 1;
-constexpr int kMaxCluster = 16;
+// must fit beside them: 5 * 32 * 96 + 32 * 32 <= 16384.
+constexpr int kFfnMaxRegs = 96;
 constexpr int kSeg = 128;                    // K elements per segment (64 code bytes)
 
 struct Group {
@@ -74,19 +72,16 @@ struct FfnArgs {
     const float* tscale;
     const uint32_t* need;
     const uint32_t* ready;
-    unsigned int* ctr;         // [0, C): per row-block group counts; abort, done
+    float* hbuf;               // [T * k][I] h of each (token, rank), fp32
+    unsigned int* ctr;         // [H/16] row tiles, [kMaxDecodePairs] groups, [kMaxDecodePairs] pair maxima,
+                               // abort flag, done count
     int T, k, H, I, E, S, layer;
-    int C;                     // CTAs per cluster
-    int RA;                    // gate (and up) rows per A stage: 16 or 32
-    int RB;                    // down rows per B stage: 16, 32, 64 or 128
+    int TRB;                   // 16-row down tiles per B stage: 1, 2, 4 or 8
     int stage_bytes, nstage;
-    int ks;                    // A: K split of a unit (1, 2, 4): 2 ks warps per unit
-    int nAU;                   // A: units at work (divides nstage)
-    int nBU;                   // B: warp groups at work (divides nstage)
     // byte offsets in dynamic shared memory
-    int o_groups, o_misc, o_red, o_hloc, o_x, o_h, o_stage;
+    int o_groups, o_misc, o_ts, o_red, o_frag, o_stage;
     unsigned long long ready_ns, dep_ns, pipe_ns;
-    unsigned long long* trace;   // optional [gridDim][16] phase stamps (ns), or null
+    unsigned long long* trace;   // optional [gridDim][32] phase stamps (ns), or null
 };
 
 // ------------------------------------------------------------------ helpers
@@ -158,73 +153,14 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// ------------------------------------------------------------- cluster plumbing
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t cluster_id_x() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t ncluster_x() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-    return r;
-}
-
-// All threads of all CTAs of the cluster (release / acquire at cluster scope).
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Address of the same shared-memory variable in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_peer(const void* p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t peer_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;"
-        " selp.u32 %0, 1, 0, p; }"
-        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ uint4 ld_peer_v4(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared::cluster.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ float ld_peer_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 // Bounded wait on an mbarrier phase that also gives up as soon as another wait
 // of the launch has raised the abort flag.
 __device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, unsigned long long limit_ns,
-                                                volatile unsigned int* abort_flag, bool cluster_scope = false) {
-    if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+                                                volatile unsigned int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (unsigned it = 0;; it++) {
-        if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if ((it & 15) == 15) {
             if (*abort_flag) return false;
             if (globaltimer() - t0 > limit_ns) return false;
@@ -232,15 +168,37 @@ __device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, 
     }
 }
 
+// Acquire at GPU scope.  The ready tickets and the slot bytes they publish are
+// this GPU's memory, written by its SM copy kernel or by its copy engine ahead of
+// a stream write of the ticket; the slot bytes are read by bulk copies through L2.
+__device__ __forceinline__ unsigned ld_acquire_gpu_u32(const unsigned int* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ bool wait_ready(const uint32_t* ready, uint32_t want, unsigned long long limit_ns,
                                            volatile unsigned int* abort_flag) {
-    if (ld_acquire_sys_u32(ready) == want) return true;
+    if (ld_acquire_gpu_u32(ready) == want) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
-        if (ld_acquire_sys_u32(ready) == want) return true;
+        if (ld_acquire_gpu_u32(ready) == want) return true;
         if (*abort_flag) return false;
         if (globaltimer() - t0 > limit_ns) return false;
         __nanosleep(64);
+    }
+}
+
+// Bounded wait (acquire) until a counter of this launch reaches `want`.
+__device__ __forceinline__ bool wait_count(const unsigned int* ctr, unsigned want, unsigned long long limit_ns,
+                                           volatile unsigned int* abort_flag) {
+    if (ld_acquire_gpu_u32(ctr) >= want) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (ld_acquire_gpu_u32(ctr) >= want) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
+        __nanosleep(32);
     }
 }
 
@@ -387,46 +345,47 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + a.nstage;
-    uint64_t* hready = empty + a.nstage;                               // [2]
     Group* groups = reinterpret_cast<Group*>(smem + a.o_groups);
     float* xinv = reinterpret_cast<float*>(smem + a.o_misc);           // [16] per token
     float* hinv = xinv + kMaxDecodeT;                                  // [16] per member
-    float* hsc = hinv + kMaxDecodeT;                                   // [16] per member
-    int* s_misc = reinterpret_cast<int*>(hsc + kMaxDecodeT);           // [8]
-    float* pairbuf = reinterpret_cast<float*>(smem + a.o_red);         // [unit][2][2 (gate, up)][ks][16][T]
-    float* hloc = reinterpret_cast<float*>(smem + a.o_hloc);           // [2][T][I/C], then [2][T] maxima
-    uint4* xf = reinterpret_cast<uint4*>(smem + a.o_x);                // x fragments, N = T
-    uint4* hf_hi = reinterpret_cast<uint4*>(smem + a.o_h);             // h fragments, N = T
+    unsigned* hmx = reinterpret_cast<unsigned*>(hinv + kMaxDecodeT);   // [16] per token (x staging)
+    int* s_misc = reinterpret_cast<int*>(hmx + kMaxDecodeT);           // [8]
+    float* ts_row = reinterpret_cast<float*>(smem + a.o_ts);           // [E][3] this layer's tensor scales
+    float* unitbuf = reinterpret_cast<float*>(smem + a.o_red);         // [unit][2][2 (gate, up)][ks][16][T]
+    uint4* xf = reinterpret_cast<uint4*>(smem + a.o_frag);             // x fragments (A), N = T
+    uint4* hf_hi = reinterpret_cast<uint4*>(smem + a.o_frag);          // h fragments (B), same bytes
     uint4* hf_lo = hf_hi + (size_t)a.T * a.I / 8;
     uint8_t* stages = smem + a.o_stage;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    volatile unsigned int* abort_flag = a.ctr + kAbortIdx;
+    const int T = a.T, H = a.H, I = a.I;
+    unsigned int* rowcnt = a.ctr;                                      // [H/16] groups done per row tile
+    unsigned int* gcnt = a.ctr + H / 16;                               // [kMaxDecodePairs] h values published
+    unsigned int* pmax = gcnt + kMaxDecodePairs;                       // [kMaxDecodePairs] max |h| bits per pair
+    volatile unsigned int* abort_flag = pmax + kMaxDecodePairs;
+    unsigned int* done_ctr = pmax + kMaxDecodePairs + 1;
     const int bs = FMT == MOE_MXFP4 ? 32 : 16;
-    const int T = a.T, H = a.H, I = a.I, C = a.C;
-    const int rho = (int)cluster_rank(), cid = (int)cluster_id_x(), ncl = (int)ncluster_x();
-    const int IC = I / C, HC = H / C;
-    const int nA = IC / a.RA, nB = HC / a.RB;               // stages per group
+    const int nTA = I / 16, nTB = H / 16;                              // A items, B tiles per group
     const int nsegA = H / kSeg, nsegB = I / kSeg;
-    const uint32_t SA = H / bs, SB = I / bs;                 // scale bytes of a gate/up row, a down row
+    const uint32_t SA = H / bs, SB = I / bs;                           // scale bytes of a gate/up row, a down row
+    const uint32_t CA = 16 * (H / 2);                                  // code bytes of 16 gate (or up) rows
     unsigned long long* trace = a.trace ? a.trace + (size_t)blockIdx.x * 32 : nullptr;
     if (trace && tid == 0) trace[0] = globaltimer();
 
     // ---- prologue 1 (may overlap the kernel before this one in the stream):
-    // barriers, and the activations, which predate the router: per-token
-    // power-of-two scale, f16 B fragments
+    // barriers, the layer's tensor scales (written only when experts are loaded
+    // into the host store), and the activations, which predate the router:
+    // per-token power-of-two scale, f16 B fragments
     if (tid == 0) {
         for (int i = 0; i < a.nstage; i++) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kNC);
         }
-        mbar_init(&hready[0], C);
-        mbar_init(&hready[1], C);
         fence_mbar_init();
     }
+    for (int i = tid; i < a.E * 3; i += blockDim.x) ts_row[i] = a.tscale[(size_t)a.layer * a.E * 3 + i];
     {
-        unsigned* tok_amax = reinterpret_cast<unsigned*>(hsc);
-        if (tid < T) tok_amax[tid] = 0u;
+        if (tid < T) hmx[tid] = 0u;
         __syncthreads();
         const int nvec = T * H / 8;
         for (int v = tid; v < nvec; v += blockDim.x) {
@@ -436,12 +395,12 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
 #pragma unroll
             for (int i = 0; i < 4; i++)
                 mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(u[i] << 16)), fabsf(__uint_as_float(u[i] & 0xFFFF0000u))));
-            atomicMax(tok_amax + (v * 8) / H, __float_as_uint(mx));
+            atomicMax(hmx + (v * 8) / H, __float_as_uint(mx));
         }
         __syncthreads();
         for (int v = tid; v < nvec; v += blockDim.x) {
             const int t = (v * 8) / H, h = v * 8 - t * H;
-            const float sc = act_scale(__uint_as_float(tok_amax[t]));
+            const float sc = act_scale(__uint_as_float(hmx[t]));
             const uint4 qv = __ldg(reinterpret_cast<const uint4*>(a.x) + v);
             const uint32_t u[4] = {qv.x, qv.y, qv.z, qv.w};
             float f[8];
@@ -455,8 +414,6 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
         }
     }
     __syncthreads();
-    // the cluster's barrier initialisations are visible before any peer arrives remotely
-    cluster_sync_all();
     if (trace && tid == 0) trace[1] = globaltimer();
 
     // ---- the slot lookup's outputs (slot_of, tickets) are needed from here on
@@ -472,69 +429,71 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     unsigned* need_s = reinterpret_cast<unsigned*>(s_s + kMaxDecodePairs);
     int* lead_s = reinterpret_cast<int*>(need_s + kMaxDecodePairs);   // first entry of my expert
     int* mi_s = lead_s + kMaxDecodePairs;                  // my index inside the group
-    int* grank_s = mi_s + kMaxDecodePairs;                 // group rank of a leader
-    int* rdy_s = grank_s + kMaxDecodePairs;                // slot shows the needed ticket
-    float* ts_s = reinterpret_cast<float*>(rdy_s + kMaxDecodePairs);   // [n][3] tensor scales
+    int* gm_s = mi_s + kMaxDecodePairs;                    // members of a leader's group
+    int* rdy_s = gm_s + kMaxDecodePairs;                   // slot shows the needed ticket
+    int* lpos_s = rdy_s + kMaxDecodePairs;                 // [leaders] entry of each leader
+    int* grank_s = lpos_s + kMaxDecodePairs;               // group rank of a leader
+    unsigned long long* lkey_s = reinterpret_cast<unsigned long long*>(grank_s + kMaxDecodePairs);  // [leaders]
     const int n = T * a.k;
+    if (tid == 0) s_misc[0] = 0;
     if (tid < n) {
         const int e = a.idx[tid], sl = a.slot_of[tid];
         int bad = 0;
         if (e < 0 || e >= a.E) bad |= MOE_STATUS_BAD_EXPERT;
         if (sl < 0 || sl >= a.S) bad |= MOE_STATUS_BAD_SLOT;
         uint32_t nd = 0u, rd = 1u;
-        float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f;
         if (!bad) {
             nd = a.need[sl];
-            rd = ld_acquire_sys_u32(a.ready + sl);
-            const float* ts = a.tscale + ((size_t)a.layer * a.E + e) * 3;
-            t0 = ts[0];
-            t1 = ts[1];
-            t2 = ts[2];
+            rd = ld_acquire_gpu_u32(a.ready + sl);
         }
         e_s[tid] = bad ? -1 : e;
         s_s[tid] = sl;
         need_s[tid] = nd;
         rdy_s[tid] = (rd == nd);
-        ts_s[3 * tid] = t0;
-        ts_s[3 * tid + 1] = t1;
-        ts_s[3 * tid + 2] = t2;
+        gm_s[tid] = 0;
         if (bad && blockIdx.x == 0) atomicOr(a.status, bad);
     }
     __syncthreads();
+    // leader (first entry of the same expert) and index among the expert's
+    // entries, by one scan of the earlier entries (broadcast loads)
     if (tid < n && e_s[tid] >= 0) {
         const int e = e_s[tid];
         int lead = tid, mi = 0;
-        for (int j = 0; j < tid; j++)
-            if (e_s[j] == e) {
-                if (lead == tid) lead = j;
-                mi++;
-            }
+#pragma unroll 8
+        for (int j = 0; j < tid; j++) {
+            const bool same = e_s[j] == e;
+            lead = same && j < lead ? j : lead;
+            mi += same;
+        }
         lead_s[tid] = lead;
         mi_s[tid] = mi;
+        atomicAdd(gm_s + lead, 1);
+        if (lead == tid) {
+            const int li = atomicAdd(s_misc, 1);
+            lkey_s[li] = ((unsigned long long)need_s[tid] << 32) | (unsigned)e;
+            lpos_s[li] = tid;
+        }
     }
     __syncthreads();
-    // leaders: rank by (ticket the slot must show, expert) so resident experts come
+    // groups ranked by (ticket the slot must show, expert): resident experts come
     // first and missed ones in the order the copy engine delivers them
-    if (tid < n && e_s[tid] >= 0 && lead_s[tid] == tid) {
-        const int e = e_s[tid];
-        const unsigned kt = need_s[tid];
-        int rank = 0, M = 0;
-        for (int j = 0; j < n; j++) {
-            const int ej = e_s[j];
-            if (ej < 0) continue;
-            if (ej == e) M++;
-            if (lead_s[j] == j && (need_s[j] < kt || (need_s[j] == kt && ej < e))) rank++;
-        }
-        grank_s[tid] = rank;
+    const int nl = s_misc[0];
+    if (tid < nl) {
+        const unsigned long long key = lkey_s[tid];
+        int rank = 0;
+#pragma unroll 8
+        for (int j = 0; j < nl; j++) rank += lkey_s[j] < key;
+        const int ld = lpos_s[tid], e = e_s[ld];
+        grank_s[ld] = rank;
         Group& G = groups[rank];
         G.expert = e;
-        G.slot = s_s[tid];
-        G.M = M;
-        G.ready = rdy_s[tid];
-        G.need = kt;
-        G.ts[0] = ts_s[3 * tid];
-        G.ts[1] = ts_s[3 * tid + 1];
-        G.ts[2] = ts_s[3 * tid + 2];
+        G.slot = s_s[ld];
+        G.M = gm_s[ld];
+        G.ready = rdy_s[ld];
+        G.need = need_s[ld];
+        G.ts[0] = ts_row[3 * e];
+        G.ts[1] = ts_row[3 * e + 1];
+        G.ts[2] = ts_row[3 * e + 2];
     }
     __syncthreads();
     if (tid < n && e_s[tid] >= 0) {
@@ -543,35 +502,38 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
         G.rank[mi_s[tid]] = (uint8_t)(tid % a.k);
         G.wt[mi_s[tid]] = a.w[tid];
     }
-    if (warp == 0) {
-        int c = 0;
-        for (int i = lane; i < n; i += 32) c += (e_s[i] >= 0 && lead_s[i] == i);
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-        if (lane == 0) s_misc[0] = c;
-    }
     __syncthreads();
     const int ng = s_misc[0];
-    if (trace && tid == 0) {
-        trace[3] = globaltimer();
-        trace[12] = (unsigned long long)((ng - cid + ncl - 1) / ncl);
-        trace[13] = (unsigned long long)C;
-        trace[14] = (unsigned long long)rho;
-    }
+    if (trace && tid == 0) trace[3] = globaltimer();
 
-    // Stage layouts (row-major, as in the slot): A = RA code rows of gate, RA of up,
-    // then their RA scale rows each; B = RB code rows of down, then their scale rows.
-    const int RA = a.RA, RB = a.RB;
-    const uint32_t CA = (uint32_t)RA * (H / 2);               // one tensor's code bytes in an A stage
-    const uint32_t CB = (uint32_t)RB * (I / 2);
+    // ---- this CTA's work: A items [a0, a1) and B tiles [b0, b1) of the call's
+    // lists (group-major, in ticket order); B stages are runs of up to TRB tiles
+    // of one group
+    const int P = gridDim.x, cta = blockIdx.x;
+    const int NAi = ng * nTA, NBt = ng * nTB;
+    const int a0 = (int)((long long)cta * NAi / P), a1 = (int)((long long)(cta + 1) * NAi / P);
+    const int b0 = (int)((long long)cta * NBt / P), b1 = (int)((long long)(cta + 1) * NBt / P);
+    const int nA = a1 - a0;
+    auto bstage = [&](int i, int& g, int& r, int& nt) {
+        g = i / nTB;
+        r = i - g * nTB;
+        nt = min(a.TRB, min(b1 - i, nTB - r));
+    };
+
     if (warp == kNC) {
         // ---------------------------------------------------------------- producer
-        const uint32_t txA = 2u * CA + 2u * RA * SA;
-        const uint32_t txB = CB + (uint32_t)RB * SB;
-        int st = 0;
+        int st = 0, issued = 0, lastg = -1;
         uint32_t round = 0;
-        int issued = 0;
-        for (int g = cid; g < ng; g += ncl) {
+        const uint8_t* blk = nullptr;
+        // first use of a group's slot: a slot that showed its ticket when the table
+        // was built was acquired then (and the CTA barrier since orders it); for a
+        // pending one, wait (bounded) for the ticket and acquire it here.  Then the
+        // bulk (async proxy) reads are ordered after the acquire.
+        fence_proxy_async_global();
+        if (trace && lane == 0) trace[9] = globaltimer();
+        auto use_group = [&](int g) {
+            if (g == lastg) return;
+            lastg = g;
             const Group& G = groups[g];
             if (!G.ready) {
                 bool ok = true;
@@ -581,41 +543,55 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
                     atomicOr(a.status, MOE_STATUS_READY_TIMEOUT);
                     *abort_flag = 1;
                 }
+                (void)ld_acquire_gpu_u32(a.ready + G.slot);
+                fence_proxy_async_global();
             }
-            // every lane acquires the ticket itself, then orders its bulk (async
-            // proxy) reads of the slot after that acquire
-            (void)ld_acquire_sys_u32(a.ready + G.slot);
-            fence_proxy_async_global();
-            const uint8_t* blk = a.slots + (unsigned long long)G.slot * a.block_bytes;
-            for (int s = 0; s < nA + nB; s++) {
-                bool ok = true;
-                if (lane == 0) ok = mbar_wait_abort(&empty[st], (round & 1) ^ 1, a.pipe_ns, abort_flag);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok && lane == 0) {
-                    atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
-                    *abort_flag = 1;
-                }
-                uint8_t* dst = stages + (size_t)st * a.stage_bytes;
-                if (lane == 0) mbar_arrive_expect_tx(&full[st], s < nA ? txA : txB);
-                __syncwarp();
-                if (s < nA) {
-                    const unsigned long long r0 = (unsigned long long)(rho * IC + RA * s);
-                    if (lane == 0) bulk_g2s(dst, blk + a.off[0] + r0 * (H / 2), CA, &full[st]);
-                    if (lane == 1) bulk_g2s(dst + CA, blk + a.off[2] + r0 * (H / 2), CA, &full[st]);
-                    if (lane == 2) bulk_g2s(dst + 2 * CA, blk + a.off[1] + r0 * SA, RA * SA, &full[st]);
-                    if (lane == 3) bulk_g2s(dst + 2 * CA + RA * SA, blk + a.off[3] + r0 * SA, RA * SA, &full[st]);
-                } else {
-                    const unsigned long long r0 = (unsigned long long)(rho * HC + (s - nA) * RB);
-                    if (lane == 0) bulk_g2s(dst, blk + a.off[4] + r0 * (I / 2), CB, &full[st]);
-                    if (lane == 1) bulk_g2s(dst + CB, blk + a.off[5] + r0 * SB, RB * SB, &full[st]);
-                }
-                if (trace && lane == 0 && issued < 8) trace[24 + issued] = globaltimer();
-                issued++;
-                if (++st == a.nstage) {
-                    st = 0;
-                    round++;
-                }
+            blk = a.slots + (unsigned long long)G.slot * a.block_bytes;
+        };
+        auto take_slot = [&](uint32_t tx) -> uint8_t* {
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait_abort(&empty[st], (round & 1) ^ 1, a.pipe_ns, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok && lane == 0) {
+                atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
+                *abort_flag = 1;
             }
+            if (lane == 0) mbar_arrive_expect_tx(&full[st], tx);
+            __syncwarp();
+            return stages + (size_t)st * a.stage_bytes;
+        };
+        auto advance = [&]() {
+            if (trace && lane == 0 && issued < 8) trace[24 + issued] = globaltimer();
+            issued++;
+            if (++st == a.nstage) {
+                st = 0;
+                round++;
+            }
+        };
+        // A item: 16 rows of gate and the same rows of up, codes then scales
+        for (int i = a0; i < a1; i++) {
+            const int g = i / nTA, t = i - g * nTA;
+            use_group(g);
+            uint8_t* dst = take_slot(2 * CA + 2 * 16 * SA);
+            const unsigned long long r0 = (unsigned long long)t * 16;
+            if (lane == 0) bulk_g2s(dst, blk + a.off[0] + r0 * (H / 2), CA, &full[st]);
+            if (lane == 1) bulk_g2s(dst + CA, blk + a.off[2] + r0 * (H / 2), CA, &full[st]);
+            if (lane == 2) bulk_g2s(dst + 2 * CA, blk + a.off[1] + r0 * SA, 16 * SA, &full[st]);
+            if (lane == 3) bulk_g2s(dst + 2 * CA + 16 * SA, blk + a.off[3] + r0 * SA, 16 * SA, &full[st]);
+            advance();
+        }
+        // B stage: nt * 16 rows of down, codes then scales
+        for (int i = b0; i < b1;) {
+            int g, r, nt;
+            bstage(i, g, r, nt);
+            i += nt;
+            use_group(g);
+            const uint32_t cb = (uint32_t)nt * 16 * (I / 2), sbb = (uint32_t)nt * 16 * SB;
+            uint8_t* dst = take_slot(cb + sbb);
+            const unsigned long long r0 = (unsigned long long)r * 16;
+            if (lane == 0) bulk_g2s(dst, blk + a.off[4] + r0 * (I / 2), cb, &full[st]);
+            if (lane == 1) bulk_g2s(dst + cb, blk + a.off[5] + r0 * SB, sbb, &full[st]);
+            advance();
         }
         if (trace && lane == 0) trace[11] = globaltimer();
         // no copy may still be in flight when the CTA exits: wait (bounded) for
@@ -626,24 +602,73 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
                     atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
     } else {
         // ---------------------------------------------------------------- consumers
-        // A stage = 16 rows of gate and the same 16 rows of up.  Unit u = warp /
-        // (2 ks) takes A stages u, u + nAU, ...: its even warps the gate tile, its
-        // odd ones the up tile, each over 1/ks of K (part kp = (warp % 2ks) / 2);
-        // the unit then sums the parts in order and forms h.
-        // B stage = RB rows of down, TRB = RB / 16 tiles: warp group warp / TRB takes
-        // B stages group, group + nBU, ..., one tile over the whole K per warp.
+        // A item = 16 rows of gate and the same 16 rows of up.  Unit u = warp /
+        // (2 ks) takes the CTA's A items u, u + nAU, ...: its even warps the gate
+        // tile, its odd ones the up tile, each over 1/ks of K (part kp); the unit
+        // then sums the parts in order, forms h and stores it to global memory,
+        // counting the values it publishes per group.
+        // B stage = up to TRB tiles of 16 down rows: a group of TRB * kb warps takes
+        // B stages group, group + nBU, ..., each tile over 1/kb of K per warp (the
+        // kb parts summed in order), once every h value of the stage's group is
+        // published.
         // nAU and nBU divide the ring size, so within a phase every slot is filled
         // and emptied for one unit (or group) only, in order: a wait never meets a
         // slot whose earlier fill is still pending (whose phase parity would
         // alias).  Consumer barriers separate the phases.
         const int g8 = lane >> 2, q = lane & 3;
-        const int ks = a.ks, uw = 2 * ks, unit = warp / uw, widx = warp - unit * uw;
-        const int role = widx & 1, kp = widx >> 1, segsA = nsegA / ks;
-        const int TRB = RB / 16, grp = warp / TRB, tile = warp % TRB;
-        const int nAU = a.nAU, nBU = a.nBU;
         const uint32_t qs = FMT == MOE_NVFP4 ? 2 * q : 0;   // the thread's scale bytes in a row's segment
         const int bstride = 4 * T;                         // pieces between the words j of a segment
-        int gi = 0, it = 0, pst = 0;                       // global stage index, group count, pair stages
+        // the K split with the fewest rounds for this CTA's A items (one round =
+        // an item's full-K dot products / ks), a little weight against more warps
+        // meeting at every item
+        int ks = 1, nAU = 1;
+        {
+            float best = 1e30f;
+            for (int c = 1; c <= kNC / 2; c *= 2) {
+                if (nsegA % c) continue;
+                int u = min(kNC / (2 * c), a.nstage);
+                while (a.nstage % u) u--;
+                const float cost = (float)((nA + u - 1) / u) / (float)c + 0.05f * (float)c;
+                if (cost < best) {
+                    best = cost;
+                    ks = c;
+                    nAU = u;
+                }
+            }
+        }
+        const int uw = 2 * ks, unit = warp / uw, widx = warp - unit * uw;
+        const int role = widx & 1, kp = widx >> 1, segsA = nsegA / ks;
+        // B: the K split kb (1, 2, 4) with the fewest rounds for this CTA's stages
+        const int TRB = a.TRB;
+        int nbst = 0;
+        for (int i = b0; i < b1; nbst++) {
+            int g, r, nt;
+            bstage(i, g, r, nt);
+            i += nt;
+        }
+        int kb = 1, nBU = 1;
+        {
+            float best = 1e30f;
+            for (int c = 1; c <= 4 && TRB * c <= kNC; c *= 2) {
+                if (nsegB % c) continue;
+                int u = min(kNC / (TRB * c), a.nstage);
+                while (a.nstage % u) u--;
+                const float cost = (float)((nbst + u - 1) / u) / (float)c + 0.05f * (float)c;
+                if (cost < best) {
+                    best = cost;
+                    kb = c;
+                    nBU = u;
+                }
+            }
+        }
+        const int gw = TRB * kb, grp = warp / gw, bw = warp - grp * gw;
+        const int tile = bw % TRB, bkp = bw / TRB, segsB = nsegB / kb;
+        if (trace && tid == 0) {
+            trace[12] = (unsigned long long)nA;
+            trace[13] = (unsigned long long)(b1 - b0);
+            trace[14] = (unsigned long long)ks;
+            trace[15] = (unsigned long long)kb;
+        }
         auto slot_wait = [&](int k) {
             if (!mbar_wait_abort(&full[k % a.nstage], (uint32_t)(k / a.nstage) & 1, a.pipe_ns, abort_flag)) {
                 if (lane == 0) atomicOr(a.status, MOE_STATUS_PIPE_TIMEOUT);
@@ -657,183 +682,223 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
                 asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;"
                              ::"r"(smem_addr(&empty[k % a.nstage])), "r"(kNC / n) : "memory");
         };
-        for (int g = cid; g < ng; g += ncl, it++) {
+        int k = 0, pst = 0;                                // stage index, unit stages done
+
+        // ---- A
+        for (int s = 0; s < nA; s++, k++) {
+            if (unit >= nAU || s % nAU != unit) continue;
+            const int i = a0 + s, g = i / nTA, t = i - g * nTA;
             const Group& G = groups[g];
-            const int M = G.M, hb = it & 1;
-            float* hl = hloc + (size_t)hb * T * IC;                        // [M][IC] this CTA's slice of h
-            unsigned* hmx = reinterpret_cast<unsigned*>(hloc + (size_t)2 * T * IC) + hb * T;   // [M] |h| max
-            if (tid < T) hmx[tid] = 0u;
-            named_sync(1, kConsThreads);     // hmx is zero before any pair adds to it
-            // this lane's B columns: member m = g8 + 8 nt of the group (null past M)
-            const uint4* xb[1][NT];            // x of the member's token
-            const uint4* hb2[2][NT];           // h of the member: high parts, remainders
+            const int M = G.M;
+            slot_wait(k);
+            if (trace && tid == 0 && s == 0) trace[4] = globaltimer();
+            if (trace && lane == 0 && widx == 0 && s < 8) trace[16 + s] = globaltimer();
+            const uint8_t* sb = stages + (size_t)(k % a.nstage) * a.stage_bytes;
+            const uint8_t* tb = sb + role * CA;                       // gate or up codes
+            const uint8_t* tsc = sb + 2 * CA + role * 16 * SA;        // their scale rows
+            const uint4* xb[1][NT];                                   // x of the member's token
 #pragma unroll
             for (int nt = 0; nt < NT; nt++) {
                 const int m = g8 + 8 * nt;
                 xb[0][nt] = m < M ? xf + (size_t)G.tok[m] * 4 + q : nullptr;
-                hb2[0][nt] = m < M ? hf_hi + (size_t)m * 4 + q : nullptr;
-                hb2[1][nt] = m < M ? hf_lo + (size_t)m * 4 + q : nullptr;
             }
-
-            // ---- A: stage s = gate rows [rho*IC + 16 s, +16) and the same rows of up
-            for (int s = 0; s < nA; s++) {
-                const int k = gi + s;
-                if (unit >= nAU || s % nAU != unit) continue;
-                slot_wait(k);
-                if (trace && tid == 0 && it == 0 && s == 0) trace[4] = globaltimer();
-                if (trace && lane == 0 && widx == 0 && it == 0 && s < 8) trace[16 + s] = globaltimer();
-                const uint8_t* sb = stages + (size_t)(k % a.nstage) * a.stage_bytes;
-                const uint8_t* tb = sb + role * CA;                       // gate or up codes
-                const uint8_t* tsc = sb + 2 * CA + role * RA * SA;        // their scale rows
-                float part[NT][4];
-                tile_mma<FMT, NT, 1>(tb + g8 * (H / 2) + 16 * q, 8 * (H / 2), tsc + g8 * SA + qs, 8 * SA, q,
-                                     kp * segsA, segsA, xb, bstride, part);
-                slot_release(k, uw);
-                // the unit's parts: [parity][role][kp][16][T]
-                float* ub = pairbuf + (size_t)unit * 2 * 2 * ks * 16 * T + (size_t)(pst & 1) * 2 * ks * 16 * T;
-                float* pb = ub + (size_t)(role * ks + kp) * 16 * T;
+            float part[NT][4];
+            tile_mma<FMT, NT, 1>(tb + g8 * (H / 2) + 16 * q, 8 * (H / 2), tsc + g8 * SA + qs, 8 * SA, q,
+                                 kp * segsA, segsA, xb, bstride, part);
+            slot_release(k, uw);
+            // the unit's parts: [parity][role][kp][16][T]
+            float* ub = unitbuf + (size_t)unit * 2 * 2 * ks * 16 * T + (size_t)(pst & 1) * 2 * ks * 16 * T;
+            float* pb = ub + (size_t)(role * ks + kp) * 16 * T;
 #pragma unroll
-                for (int nt = 0; nt < NT; nt++)
+            for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        const int rr = g8 + (e >> 1) * 8, m = 8 * nt + 2 * q + (e & 1);
-                        if (m < M) pb[rr * T + m] = part[nt][e];
-                    }
-                named_sync(2 + unit, 32 * uw);
-                for (int o = widx * 32 + lane; o < 16 * M; o += 32 * uw) {
-                    const int rr = o & 15, m = o >> 4;
+                for (int e = 0; e < 4; e++) {
+                    const int rr = g8 + (e >> 1) * 8, m = 8 * nt + 2 * q + (e & 1);
+                    if (m < M) pb[rr * T + m] = part[nt][e];
+                }
+            named_sync(2 + unit, 32 * uw);
+            int cnt = 0;
+            // o = 16 m + row: each half-warp holds the 16 rows of one member
+            for (int base = widx * 32; base < 16 * M; base += 32 * uw) {
+                const int o = base + lane, rr = o & 15, m = o >> 4;
+                float hv = 0.0f;
+                int pair = 0;
+                if (o < 16 * M) {
                     float gs = ub[rr * T + m], us = ub[(size_t)ks * 16 * T + rr * T + m];
                     for (int p = 1; p < ks; p++) {
                         gs += ub[(size_t)p * 16 * T + rr * T + m];
                         us += ub[(size_t)(ks + p) * 16 * T + rr * T + m];
                     }
-                    const float xs = xinv[G.tok[m]];                   // undo x's scale
+                    const float xs = xinv[G.tok[m]];               // undo x's scale
                     const float gv = gs * xs * G.ts[0], uv = us * xs * G.ts[1];
-                    const float hv = gv / (1.0f + expf(-gv)) * uv;
-                    hl[m * IC + s * 16 + rr] = hv;
-                    atomicMax(hmx + m, __float_as_uint(fabsf(hv)));
+                    hv = gv / (1.0f + expf(-gv)) * uv;
+                    pair = G.tok[m] * a.k + G.rank[m];
+                    a.hbuf[(size_t)pair * I + t * 16 + rr] = hv;
+                    cnt++;
                 }
-                pst++;
-            }
-            gi += nA;
-            named_sync(1, kConsThreads);     // every row of this CTA's slice of h is written
-            if (trace && tid == 0 && it == 0) trace[5] = globaltimer();
-
-            // ---- X: publish the slice to every CTA of the cluster (itself included),
-            // wait until all have published, gather the whole h
-            // lane p arrives on peer p's barrier (the release fences run side by side)
-            if (tid < C) mbar_arrive_remote(map_peer(&hready[hb], (uint32_t)tid));
-            if (!mbar_wait_abort(&hready[hb], (uint32_t)(it >> 1) & 1, a.dep_ns, abort_flag, true)) {
-                if (lane == 0) atomicOr(a.status, MOE_STATUS_DEP_TIMEOUT);
-                *abort_flag = 1;
-            }
-            if (trace && tid == 0 && it == 0) trace[6] = globaltimer();
-            if (tid < M) {
-                float mx = 0.0f;
-                for (int p = 0; p < C; p++) mx = fmaxf(mx, ld_peer_f32(map_peer(hmx + tid, (uint32_t)p)));
-                const float sc = act_scale(mx);
-                hsc[tid] = sc;
-                hinv[tid] = 1.0f / sc;
-            }
-            named_sync(1, kConsThreads);
-            for (int v = tid; v < M * (I / 8); v += kConsThreads) {
-                const int m = v / (I / 8), k0 = (v - m * (I / 8)) * 8;
-                const int p = k0 / IC, il = k0 - p * IC;
-                const uint32_t src = map_peer(hl + m * IC + il, (uint32_t)p);
-                const uint4 u0 = ld_peer_v4(src), u1 = ld_peer_v4(src + 16);
-                const float sc = hsc[m];
-                const float hv[8] = {__uint_as_float(u0.x) * sc, __uint_as_float(u0.y) * sc,
-                                     __uint_as_float(u0.z) * sc, __uint_as_float(u0.w) * sc,
-                                     __uint_as_float(u1.x) * sc, __uint_as_float(u1.y) * sc,
-                                     __uint_as_float(u1.z) * sc, __uint_as_float(u1.w) * sc};
-                float hi[8], lo[8];
+                float mx = fabsf(hv);
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    hi[i] = __half2float(__float2half_rn(hv[i]));
-                    lo[i] = hv[i] - hi[i];                 // exact in fp32
-                }
-                const int pi = piece_index(k0, m, T);
-                hf_hi[pi] = pack_piece(hi);
-                hf_lo[pi] = pack_piece(lo);
+                for (int off = 8; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                if ((lane & 15) == 0 && o < 16 * M) atomicMax(pmax + pair, __float_as_uint(mx));
             }
-            named_sync(1, kConsThreads);
-            if (trace && tid == 0 && it == 0) trace[7] = globaltimer();
+            // publish: the warp's h values and maxima are visible before the group's count grows
+            cnt = __reduce_add_sync(0xffffffffu, cnt);
+            __syncwarp();
+            if (lane == 0 && cnt) {
+                __threadfence();
+                atomicAdd(gcnt + g, (unsigned)cnt);
+            }
+            pst++;
+        }
+        named_sync(1, kConsThreads);      // x fragments are dead from here on
+        if (trace && tid == 0) trace[5] = globaltimer();
 
-            // ---- B: stage b = down rows [rho*HC + RB b, +RB); warp `tile` of group b % ngrp
-            for (int b = 0; b < nB; b++) {
-                const int k = gi + b;
-                if (b % nBU != grp) continue;
-                slot_wait(k);
-                if (trace && lane == 0 && tile == 0 && it == 0 && nA + b < 8) trace[16 + nA + b] = globaltimer();
+        // ---- B
+        int curg = -1, nbs = 0, bps = 0;
+        const uint4* hb2[2][NT] = {};     // h of the member: high parts, remainders
+        for (int i = b0; i < b1; nbs++, k++) {
+            int g, r, nt;
+            bstage(i, g, r, nt);
+            i += nt;
+            const Group& G = groups[g];
+            const int M = G.M;
+            if (g != curg) {
+                // a new group: every warp is done with the previous fragments; wait
+                // (bounded) until all I * M values of its h (and their maxima) are
+                // published, then scale each member's h by a power of two and split
+                // it into f16 high parts and remainders
+                curg = g;
+                named_sync(1, kConsThreads);
+                if (tid == 0) {
+                    if (!wait_count(gcnt + g, (unsigned)(I * M), a.dep_ns, abort_flag)) {
+                        atomicOr(a.status, MOE_STATUS_DEP_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    if (trace && nbs == 0) trace[6] = globaltimer();
+                }
+                named_sync(1, kConsThreads);
+                if (tid < M) hinv[tid] = 1.0f / act_scale(__uint_as_float(__ldcg(pmax + G.tok[tid] * a.k + G.rank[tid])));
+                for (int v = tid; v < M * (I / 8); v += kConsThreads) {
+                    const int m = v / (I / 8), k0 = (v - m * (I / 8)) * 8;
+                    const int pair = G.tok[m] * a.k + G.rank[m];
+                    const float4* src = reinterpret_cast<const float4*>(a.hbuf + (size_t)pair * I + k0);
+                    const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
+                    const float sc = act_scale(__uint_as_float(__ldcg(pmax + pair)));
+                    const float hv[8] = {u0.x * sc, u0.y * sc, u0.z * sc, u0.w * sc,
+                                         u1.x * sc, u1.y * sc, u1.z * sc, u1.w * sc};
+                    float hi[8], lo[8];
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        hi[j] = __half2float(__float2half_rn(hv[j]));
+                        lo[j] = hv[j] - hi[j];                 // exact in fp32
+                    }
+                    const int pi = piece_index(k0, m, T);
+                    hf_hi[pi] = pack_piece(hi);
+                    hf_lo[pi] = pack_piece(lo);
+                }
+                named_sync(1, kConsThreads);
+                if (trace && tid == 0 && nbs == 0) trace[7] = globaltimer();
+#pragma unroll
+                for (int n8 = 0; n8 < NT; n8++) {
+                    const int m = g8 + 8 * n8;
+                    hb2[0][n8] = m < M ? hf_hi + (size_t)m * 4 + q : nullptr;
+                    hb2[1][n8] = m < M ? hf_lo + (size_t)m * 4 + q : nullptr;
+                }
+            }
+            if (grp >= nBU || nbs % nBU != grp) continue;
+            slot_wait(k);
+            if (trace && lane == 0 && bw == 0 && nA + nbs < 8) trace[16 + nA + nbs] = globaltimer();
+            float acc[NT][4];
+            if (tile < nt) {
                 const uint8_t* sb = stages + (size_t)(k % a.nstage) * a.stage_bytes;
+                const uint32_t cb = (uint32_t)nt * 16 * (I / 2);
                 const int row = tile * 16 + g8;
-                float acc[NT][4];
-                tile_mma<FMT, NT, 2>(sb + row * (I / 2) + 16 * q, 8 * (I / 2), sb + CB + row * SB + qs, 8 * SB, q,
-                                     0, nsegB, hb2, bstride, acc);
-                slot_release(k, TRB);
-                const int r0 = rho * HC + b * RB + tile * 16;
+                tile_mma<FMT, NT, 2>(sb + row * (I / 2) + 16 * q, 8 * (I / 2), sb + cb + row * SB + qs, 8 * SB, q,
+                                     bkp * segsB, segsB, hb2, bstride, acc);
+            }
+            slot_release(k, gw);    // every warp of the group arrives, with a tile or without
+            if (kb > 1) {
+                // the group's parts: [parity][tile][kp][16][T]; part 0's warp sums them
+                float* gb = unitbuf + ((size_t)grp * 2 + (bps & 1)) * TRB * kb * 16 * T;
+                if (tile < nt) {
 #pragma unroll
-                for (int nt = 0; nt < NT; nt++)
+                    for (int n8 = 0; n8 < NT; n8++)
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const int rr = g8 + (e >> 1) * 8, m = 8 * n8 + 2 * q + (e & 1);
+                            if (m < M) gb[((size_t)(tile * kb + bkp) * 16 + rr) * T + m] = acc[n8][e];
+                        }
+                }
+                named_sync(2 + grp, 32 * gw);
+                bps++;
+                if (bkp != 0 || tile >= nt) continue;
+#pragma unroll
+                for (int n8 = 0; n8 < NT; n8++)
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
-                        const int rr = g8 + (e >> 1) * 8, m = 8 * nt + 2 * q + (e & 1);
-                        if (m < M)
-                            a.y_part[((size_t)G.tok[m] * a.k + G.rank[m]) * H + r0 + rr] =
-                                G.wt[m] * (acc[nt][e] * hinv[m] * G.ts[2]);
+                        const int rr = g8 + (e >> 1) * 8, m = 8 * n8 + 2 * q + (e & 1);
+                        if (m < M) {
+                            float v = gb[((size_t)(tile * kb) * 16 + rr) * T + m];
+                            for (int p2 = 1; p2 < kb; p2++) v += gb[((size_t)(tile * kb + p2) * 16 + rr) * T + m];
+                            acc[n8][e] = v;
+                        }
                     }
+            } else if (tile >= nt) {
+                continue;
             }
-            gi += nB;
-
-            // ---- this group's rows of block rho are in y_part: count it; the last
-            // group to finish the block sums it over the ranks (K5)
-            named_sync(1, kConsThreads);
-            if (trace && tid == 0 && it == 0) trace[8] = globaltimer();
-            if (tid == 0) {
-                __threadfence();
-                const unsigned prev = atomicAdd(a.ctr + rho, 1u);
-                s_misc[1] = (prev == (unsigned)ng - 1u);
-                if (s_misc[1]) __threadfence();
-            }
-            named_sync(1, kConsThreads);
-            if (s_misc[1]) {
-                // y = the rank-ordered sum of y_part, rounded to bf16
-                const int q4 = HC / 4;
-                for (int v = tid; v < T * q4; v += kConsThreads) {
-                    const int t = v / q4, r = rho * HC + (v - t * q4) * 4;
-                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int j = 0; j < a.k; j++) {
-                        const float4 pv = __ldcg(reinterpret_cast<const float4*>(a.y_part + ((size_t)t * a.k + j) * H + r));
-                        sum.x += pv.x;
-                        sum.y += pv.y;
-                        sum.z += pv.z;
-                        sum.w += pv.w;
-                    }
-                    if (a.y) {
-                        const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(sum.x));
-                        const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(sum.y));
-                        const uint32_t b2 = __bfloat16_as_ushort(__float2bfloat16_rn(sum.z));
-                        const uint32_t b3 = __bfloat16_as_ushort(__float2bfloat16_rn(sum.w));
-                        *reinterpret_cast<uint2*>(a.y + (size_t)t * H + r) = make_uint2(b0 | (b1 << 16), b2 | (b3 << 16));
-                    }
+            const int rt = r + tile;                                   // row tile of H
+#pragma unroll
+            for (int n8 = 0; n8 < NT; n8++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int rr = g8 + (e >> 1) * 8, m = 8 * n8 + 2 * q + (e & 1);
+                    if (m < M)
+                        a.y_part[((size_t)G.tok[m] * a.k + G.rank[m]) * H + rt * 16 + rr] =
+                            G.wt[m] * (acc[n8][e] * hinv[m] * G.ts[2]);
                 }
-                if (tid == 0) a.ctr[rho] = 0u;
+            if (!a.y) continue;
+            // the row tile's part from this group is in y_part: count it; the warp
+            // that lands the last group sums the tile over the ranks in rank order
+            // and writes its bf16 rows (K5)
+            __syncwarp();
+            unsigned prev = 0;
+            if (lane == 0) {
+                __threadfence();
+                prev = atomicAdd(rowcnt + rt, 1u);
+                if (prev == (unsigned)ng - 1u) __threadfence();
             }
-            if (trace && tid == 0) trace[9] = globaltimer();
+            prev = __shfl_sync(0xffffffffu, prev, 0);
+            __syncwarp();                  // the lanes' loads below follow lane 0's fence
+            if (prev == (unsigned)ng - 1u) {
+                for (int v = lane; v < T * 16; v += 32) {
+                    const int t = v >> 4, row = rt * 16 + (v & 15);
+                    float sum = 0.0f;
+                    for (int j = 0; j < a.k; j++) sum += __ldcg(a.y_part + ((size_t)t * a.k + j) * H + row);
+                    a.y[(size_t)t * H + row] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+                }
+            }
         }
+        if (trace && tid == 0) trace[8] = globaltimer();
     }
 
-    // ---- epilogue: no CTA leaves while a peer may still read its shared memory;
-    // the last CTA clears the abort flag for the next launch
+    // ---- epilogue: the last CTA to finish clears the launch's counters and the
+    // abort flag for the next launch (every other CTA is done with them)
     __syncthreads();
-    cluster_sync_all();
     if (trace && tid == 0) trace[10] = globaltimer();
     if (tid == 0) {
         __threadfence();
-        const unsigned int prev = atomicAdd(a.ctr + kDoneIdx, 1u);
-        if (prev == gridDim.x - 1) {
-            __threadfence();
-            a.ctr[kAbortIdx] = 0;
-            a.ctr[kDoneIdx] = 0;
+        const unsigned int prev = atomicAdd(done_ctr, 1u);
+        s_misc[2] = prev == gridDim.x - 1;
+        if (s_misc[2]) __threadfence();
+    }
+    __syncthreads();
+    if (s_misc[2]) {
+        for (int i = tid; i < H / 16; i += blockDim.x) rowcnt[i] = 0u;
+        for (int i = tid; i < 2 * kMaxDecodePairs; i += blockDim.x) gcnt[i] = 0u;   // counts and maxima
+        __syncthreads();
+        if (tid == 0) {
+            *abort_flag = 0u;
+            *done_ctr = 0u;
             __threadfence();
         }
     }
@@ -894,192 +959,84 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
 
 static size_t up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
-// Shared-memory layout and stage sizes of one launch.  A CTA streams at HBM rate
-// only with several stages in flight, so stages are small: RA = 16 gate (and up)
-// rows per A stage (one 16-row tile of each); RB = the most down rows
-// (128, 64, 32 or 16, dividing H/C) whose stage is no larger than an A stage.
-// MOE_EINVAL if not even two stages fit.
-static int plan_ffn(const moe_pool* p, int T, int C, int NT, FfnArgs& a, size_t& smem) {
+// Shared-memory layout, ring and B stage shape of a launch with T tokens.
+static int plan_ffn(const moe_pool* p, int T, FfnArgs& a, size_t& smem) {
     const moe_config& c = p->cfg;
     const int bs = p->bs;
-    const int IC = c.I / C, HC = c.H / C;
     const size_t SA = c.H / bs, SB = c.I / bs;
     const size_t budget = (size_t)p->ffn_smem;
-    {
-        const int RA = 16;
-        const size_t stA = 2 * (size_t)RA * (c.H / 2) + 2 * (size_t)RA * SA;
-        int RB = 16;
-        for (int rb = 128; rb >= 16; rb >>= 1)
-            if (HC % rb == 0 && (size_t)rb * (c.I / 2 + SB) <= std::max<size_t>(stA, (size_t)16 * (c.I / 2 + SB))) {
-                RB = rb;
-                break;
-            }
-        a.RA = RA;
-        a.RB = RB;
-        const size_t stB = (size_t)RB * (c.I / 2 + SB);
-        a.stage_bytes = (int)up(std::max(stA, stB), 128);
-        size_t o = up((2 * 16 + 2) * sizeof(uint64_t), 128);
-        a.o_groups = (int)o;
-        o += sizeof(Group) * kMaxDecodePairs;
-        a.o_misc = (int)up(o, 16);
-        o = a.o_misc + 3 * kMaxDecodeT * sizeof(float) + 8 * sizeof(int);
-        a.o_red = (int)up(o, 16);
-        o = a.o_red + (size_t)(kNC / 2) * 2 * 2 * 16 * T * sizeof(float);   // units * ks <= 4
-        a.o_hloc = (int)up(o, 16);
-        o = a.o_hloc + ((size_t)2 * T * IC + 2 * T) * sizeof(float);
-        a.o_x = (int)up(o, 16);
-        o = a.o_x + (size_t)T * c.H * 2;
-        a.o_h = (int)up(o, 16);
-        o = a.o_h + (size_t)2 * T * c.I * 2;
-        a.o_stage = (int)up(o, 128);
-        // the prologue keeps its per-(token, rank) table (7 ints + 3 floats each) in the ring
-        const size_t need_ring = std::max((size_t)2 * a.stage_bytes, (size_t)10 * 4 * kMaxDecodePairs);
-        if (a.o_stage + need_ring > budget)
-            return fail(MOE_EINVAL, "decode FFN: T * (H + 2 I) too large for shared memory (lower max_tokens)");
-        a.nstage = (int)std::min<size_t>(8, (budget - a.o_stage) / a.stage_bytes);
-        if (a.nstage >= kNC / 2) a.nstage = a.nstage / (kNC / 2) * (kNC / 2);
-        smem = a.o_stage + (size_t)a.nstage * a.stage_bytes;
-        // A: units of 2 ks warps, as many as divide the ring; the K split with the
-        // fewest rounds (one round = one stage's full-K dot products / ks) wins,
-        // a little weight against more warps meeting at every stage
-        const int nA = IC / RA, nsegA = c.H / 128;
-        double best = 1e30;
-        for (int ks = 1; ks <= kNC / 2; ks *= 2) {
-            if (nsegA % ks) continue;
-            int u = std::min(kNC / (2 * ks), a.nstage);
-            while (a.nstage % u) u--;
-            const double cost = (double)((nA + u - 1) / u) / ks + 0.05 * ks;
-            if (cost < best) {
-                best = cost;
-                a.ks = ks;
-                a.nAU = u;
-            }
+    const size_t stA = 2 * (size_t)16 * (c.H / 2) + 2 * (size_t)16 * SA;
+    const size_t rowB = c.I / 2 + SB;
+    // B stages: the most 16-row tiles (8, 4, 2 or 1) that fit an A stage (or one tile)
+    a.TRB = 1;
+    for (int t = 8; t >= 1; t >>= 1)
+        if ((size_t)t * 16 * rowB <= std::max(stA, 16 * rowB)) {
+            a.TRB = t;
+            break;
         }
-        // B: groups of RB / 16 warps, as many as divide the ring
-        a.nBU = 1;
-        for (int d = kNC / (a.RB / 16); d >= 1; d--)
-            if (a.nstage % d == 0) {
-                a.nBU = d;
-                break;
-            }
-        return MOE_OK;
-    }
-}
-
-// For every cluster size C in {16, 8, 4, 2, 1} that splits I and H into 16-row
-// tiles: how many clusters of C CTAs (with this kernel's shared memory) the GPU
-// can hold at once (0 when C does not split the shapes or no cluster fits).
-template <int FMT, int NT>
-static int query_clusters(moe_pool* p, int (&ncl)[5]) {
-    auto kern = ffn_decode_kernel<FMT, NT>;
-    const moe_config& c = p->cfg;
-    MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p->ffn_smem));
-    MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-    int any = 0;
-    cudaError_t last = cudaSuccess;
-    for (int ci = 0, C = kMaxCluster; ci < 5; ci++, C >>= 1) {
-        ncl[ci] = 0;
-        if (c.I % (16 * C) || c.H % (16 * C)) continue;
-        int n = 0;
-        if (C == 1) {
-            // a "cluster" of one CTA: plain occupancy
-            int per_sm = 0;
-            last = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFfnThreads, p->ffn_smem);
-            if (last == cudaSuccess) n = per_sm * p->num_sms;
-        } else {
-            cudaLaunchConfig_t lc = {};
-            lc.gridDim = dim3(C);
-            lc.blockDim = dim3(kFfnThreads);
-            lc.dynamicSmemBytes = p->ffn_smem;
-            cudaLaunchAttribute at[1];
-            at[0].id = cudaLaunchAttributeClusterDimension;
-            at[0].val.clusterDim.x = C;
-            at[0].val.clusterDim.y = 1;
-            at[0].val.clusterDim.z = 1;
-            lc.attrs = at;
-            lc.numAttrs = 1;
-            last = cudaOccupancyMaxActiveClusters(&n, kern, &lc);
-        }
-        if (last != cudaSuccess) {
-            (void)cudaGetLastError();
-            n = 0;
-        }
-        ncl[ci] = n;
-        any |= n > 0;
-    }
-    if (!any)
-        return fail(MOE_EINVAL, std::string("decode FFN: no cluster size fits on this GPU (last query: ") +
-                                    cudaGetErrorString(last) + ")");
+    a.stage_bytes = (int)up(std::max(stA, (size_t)a.TRB * 16 * rowB), 128);
+    size_t o = up((2 * 8) * sizeof(uint64_t), 128);
+    a.o_groups = (int)o;
+    o += sizeof(Group) * std::min(kMaxDecodePairs, c.max_tokens * c.k);
+    a.o_misc = (int)up(o, 16);
+    o = a.o_misc + 3 * kMaxDecodeT * sizeof(float) + 8 * sizeof(int);
+    a.o_ts = (int)up(o, 16);
+    o = a.o_ts + (size_t)c.E * 3 * sizeof(float);
+    a.o_red = (int)up(o, 16);
+    o = a.o_red + (size_t)(kNC / 2) * 2 * 2 * 16 * T * sizeof(float);   // units * ks <= kNC / 2
+    a.o_frag = (int)up(o, 16);
+    o = a.o_frag + std::max((size_t)T * c.H * 2, (size_t)2 * T * c.I * 2);
+    a.o_stage = (int)up(o, 128);
+    // the prologue keeps its per-(token, rank) table (9 ints + a u64 each) in the ring
+    const size_t need_ring = std::max((size_t)2 * a.stage_bytes, (size_t)11 * 4 * kMaxDecodePairs);
+    if (a.o_stage + need_ring > budget)
+        return fail(MOE_EINVAL, "decode FFN: T * H too large for shared memory (lower max_tokens)");
+    // a power of two (at most 8), so that 2, 4 or 8 consumer units can share the ring
+    const int fit = (int)std::min<size_t>(8, (budget - a.o_stage) / a.stage_bytes);
+    a.nstage = 1;
+    while (a.nstage * 2 <= fit) a.nstage *= 2;
+    smem = a.o_stage + (size_t)a.nstage * a.stage_bytes;
     return MOE_OK;
 }
 
-// The cluster size of a launch with at most `groups` unique experts.  A CTA's
-// share of a group is 1/C of it, and the clusters that fit at once take the
-// groups in ceil(groups / clusters) rounds, so the time goes as rounds / C: pick
-// the smallest, then the fewest rounds, then the larger C.
-static int g_force_cluster = 0;   // moe_set_ffn_cluster: 0 = automatic
-
-// Cluster size C of a launch: the work of one expert is split over C CTAs, and
-// the clusters that fit at once take the G unique experts in ceil(G / clusters)
-// rounds, so the time goes as rounds * (1 / C + the fixed cost of a group, about
-// 4 % of an expert on one CTA).  G is the expected number of unique experts,
-// E (1 - (1 - k/E)^T) (at most T * k).
-static void choose_cluster(const moe_pool* p, const int (&ncl)[5], int T, int& C, int& nclusters) {
-    const moe_config& c = p->cfg;
-    const double Gd = c.E * (1.0 - std::pow(1.0 - (double)c.k / c.E, (double)T));
-    const int G = std::max(1, std::min(T * c.k, (int)(Gd + 0.5)));
-    double best = 1e30;
-    C = 1;
-    nclusters = 1;
-    for (int ci = 0, cc = kMaxCluster; ci < 5; ci++, cc >>= 1) {
-        if (ncl[ci] <= 0) continue;
-        if (g_force_cluster && cc != g_force_cluster) continue;
-        const int n = std::min(ncl[ci], G);
-        const int rounds = (G + n - 1) / n;
-        const double cost = rounds * (1.0 / cc + 0.04);
-        if (cost < best - 1e-12) {
-            best = cost;
-            C = cc;
-            nclusters = std::min(ncl[ci], T * c.k);
-        }
-    }
-}
-
+// One CTA per SM; every CTA must be resident at once (B tiles wait for A items
+// of other CTAs), so the grid is what the occupancy calculator allows.
 template <int FMT, int NT>
-static int ffn_shape(moe_pool* p, FfnArgs& a, size_t& smem, int& nclusters) {
-    const int fi = FMT == MOE_NVFP4 ? 1 : 0, ni = NT - 1;
-    if (!p->ffn_attr_set[fi][ni]) {
-        int rc = query_clusters<FMT, NT>(p, p->ffn_ncl[fi][ni]);
-        if (rc) return rc;
-        p->ffn_attr_set[fi][ni] = 1;
+static int ffn_grid(moe_pool* p, int& grid) {
+    auto kern = ffn_decode_kernel<FMT, NT>;
+    const int fi = FMT == MOE_NVFP4, ni = NT - 1;
+    if (!p->ffn_grid[fi][ni]) {
+        MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p->ffn_smem));
+        int per_sm = 0;
+        MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFfnThreads, p->ffn_smem));
+        if (per_sm < 1) return fail(MOE_ECUDA, "decode FFN: no CTA fits on an SM");
+        p->ffn_grid[fi][ni] = p->num_sms;   // one per SM: more would only wait
     }
-    choose_cluster(p, p->ffn_ncl[fi][ni], a.T, a.C, nclusters);
-    return plan_ffn(p, a.T, a.C, NT, a, smem);
+    grid = p->ffn_grid[fi][ni];
+    return MOE_OK;
 }
 
 template <int FMT, int NT>
 static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     size_t smem = 0;
-    int ncl = 0;
-    int rc = ffn_shape<FMT, NT>(p, a, smem, ncl);
+    int grid = 0;
+    int rc = ffn_grid<FMT, NT>(p, grid);
+    if (rc) return rc;
+    rc = plan_ffn(p, a.T, a, smem);
     if (rc) return rc;
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(ncl * a.C);
+    lc.gridDim = dim3(grid);
     lc.blockDim = dim3(kFfnThreads);
     lc.dynamicSmemBytes = smem;
     lc.stream = s;
-    cudaLaunchAttribute at[2];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = a.C;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute at[1];
     // programmatic serialisation: the activations are staged while the slot
     // lookup before this kernel finishes (the kernel waits for it before reading
     // slot_of, the tickets and the tensor scales)
-    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[1].val.programmaticStreamSerializationAllowed = 1;
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = at;
-    lc.numAttrs = 2;
+    lc.numAttrs = 1;
     MOE_CUDA_TRY(cudaLaunchKernelEx(&lc, ffn_decode_kernel<FMT, NT>, a));
     return MOE_OK;
 }
@@ -1109,30 +1066,22 @@ extern "C" int moe_set_ffn_trace(void* buf) {
     return MOE_OK;
 }
 
-extern "C" int moe_set_ffn_cluster(int cluster) {
-    if (cluster != 0 && cluster != 1 && cluster != 2 && cluster != 4 && cluster != 8 && cluster != 16)
-        return fail(MOE_EINVAL, "cluster size must be 0 (automatic), 1, 2, 4, 8 or 16");
-    g_force_cluster = cluster;
-    return MOE_OK;
-}
-
-extern "C" int moe_ffn_launch_info(moe_pool* p, int T, int* cluster, int* clusters, int* nstage,
-                                   int* smem_bytes) {
-    if (!p || !cluster || !clusters || !nstage || !smem_bytes) return fail(MOE_EINVAL, "null argument");
+extern "C" int moe_ffn_launch_info(moe_pool* p, int T, int* ctas, int* nstage, int* stage_bytes, int* smem_bytes) {
+    if (!p || !ctas || !nstage || !stage_bytes || !smem_bytes) return fail(MOE_EINVAL, "null argument");
     if (T <= 0 || T > p->cfg.max_tokens) return fail(MOE_EINVAL, "T must be in [1, max_tokens]");
     FfnArgs a{};
-    a.T = T;
-    a.k = p->cfg.k;
     size_t smem = 0;
-    int ncl = 0, rc;
+    int grid = 0, rc;
     if (p->cfg.fmt == MOE_NVFP4)
-        rc = T <= 8 ? ffn_shape<MOE_NVFP4, 1>(p, a, smem, ncl) : ffn_shape<MOE_NVFP4, 2>(p, a, smem, ncl);
+        rc = T <= 8 ? ffn_grid<MOE_NVFP4, 1>(p, grid) : ffn_grid<MOE_NVFP4, 2>(p, grid);
     else
-        rc = T <= 8 ? ffn_shape<MOE_MXFP4, 1>(p, a, smem, ncl) : ffn_shape<MOE_MXFP4, 2>(p, a, smem, ncl);
+        rc = T <= 8 ? ffn_grid<MOE_MXFP4, 1>(p, grid) : ffn_grid<MOE_MXFP4, 2>(p, grid);
     if (rc) return rc;
-    *cluster = a.C;
-    *clusters = ncl;
+    rc = plan_ffn(p, T, a, smem);
+    if (rc) return rc;
+    *ctas = grid;
     *nstage = a.nstage;
+    *stage_bytes = a.stage_bytes;
     *smem_bytes = (int)smem;
     return MOE_OK;
 }
@@ -1169,6 +1118,7 @@ extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T,
     a.need = p->need;
     a.ready = p->ready;
     a.ctr = p->ctr;
+    a.hbuf = p->hbuf;
     a.T = T;
     a.k = c.k;
     a.H = c.H;

@@ -87,6 +87,7 @@ extern "C" int moe_pool_destroy(moe_pool* p) {
     cudaFree(p->ready);
     cudaFree(p->tscale);
     cudaFree(p->ctr);
+    cudaFree(p->hbuf);
     if (p->host) cudaFreeHost(p->host);
     if (p->lk_h) cudaFreeHost(p->lk_h);
     if (p->lk_event) cudaEventDestroy(p->lk_event);
@@ -135,7 +136,8 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
     ALLOC(p->need, S * sizeof(uint32_t));
     ALLOC(p->ready, S * sizeof(uint32_t));
     ALLOC(p->tscale, LE * 3 * sizeof(float));
-    ALLOC(p->ctr, (kMaxDecodePairs + 8) * sizeof(unsigned int));
+    ALLOC(p->ctr, ((size_t)cfg->H / 16 + 2 * kMaxDecodePairs + 8) * sizeof(unsigned int));
+    ALLOC(p->hbuf, (size_t)kMaxDecodePairs * cfg->I * sizeof(float));
 #undef ALLOC
     cudaMemset(p->slot_key, 0xFF, S * sizeof(int32_t));
     cudaMemset(p->slot_clock, 0, S * sizeof(unsigned long long));
@@ -145,7 +147,7 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
     cudaMemset(p->need, 0, S * sizeof(uint32_t));
     cudaMemset(p->ready, 0, S * sizeof(uint32_t));
     cudaMemset(p->tscale, 0, LE * 3 * sizeof(float));
-    cudaMemset(p->ctr, 0, (kMaxDecodePairs + 8) * sizeof(unsigned int));
+    cudaMemset(p->ctr, 0, ((size_t)cfg->H / 16 + 2 * kMaxDecodePairs + 8) * sizeof(unsigned int));
     e = cudaHostAlloc((void**)&p->host, host_bytes, cudaHostAllocMapped);
     if (e != cudaSuccess) {
         p->host = nullptr;

@@ -63,7 +63,7 @@ enum {
 /* Bits of the device status word written by moe_expert_ffn. */
 enum {
     MOE_STATUS_READY_TIMEOUT = 1,  /* a missed expert's ready flag never arrived */
-    MOE_STATUS_DEP_TIMEOUT = 2,    /* waited too long for the cluster's slices of h */
+    MOE_STATUS_DEP_TIMEOUT = 2,    /* waited too long for an expert's h (other CTAs) */
     MOE_STATUS_BAD_SLOT = 4,       /* slot index outside the pool */
     MOE_STATUS_BAD_EXPERT = 8,     /* expert index outside [0, E) */
     MOE_STATUS_PIPE_TIMEOUT = 16   /* a shared-memory pipeline wait gave up */
@@ -256,52 +256,49 @@ int moe_pool_set_copy_mode(moe_pool* pool, int mode);
  * values (about 22 significant bits).  If y_bf16 is not NULL the call also does
  * the combine: y_bf16[t, :] = bf16(sum over j = 0..k-1 of y_part[t, j, :]),
  * summed in fp32 in rank order, round to nearest even (the same as moe_combine).
- * One thread-block cluster per unique expert computes it (gate/up rows split
- * over the cluster's CTAs, h exchanged through distributed shared memory, down
- * rows split again); CTAs wait only for CTAs of their own cluster and for the
- * ready tickets of missed experts.  It is a plain launch with programmatic
+ * One CTA per SM computes it: CTA c takes the c-th share of the call's 16-row
+ * gate/up tiles (all unique experts, ticket order) and then of its 16-row down
+ * tiles; h goes through a pool-owned global buffer with a count per expert, and
+ * down tiles wait (bounded) for their expert's count.  All CTAs are resident at
+ * once and gate/up tiles wait only for their own copies and for the ready
+ * tickets of missed experts, so every wait ends.  Calls on one pool must not
+ * run concurrently (they share the buffer and the counts).  It is a plain launch with programmatic
  * stream serialisation: it stages x while the kernel before it (the slot lookup)
  * finishes, so x must be complete before that kernel starts (it is, when the
  * router ran on x first).  Waits are bounded (moe_set_wait_limits); failures set
  * bits of *status (device int, caller-zeroed; MOE_STATUS_*).  y_part is [T, k, H]
  * fp32, y_bf16 [T, H]; x, y_part and y_bf16 16-byte aligned.  Limits: T <=
- * max_tokens of the pool, and T * (H + 2 I) * 2 bytes of activations must fit in
- * shared memory beside two weight stages (MOE_EINVAL otherwise).
+ * max_tokens of the pool, and max(T * H, 2 * T * I) * 2 bytes of activation
+ * fragments must fit in shared memory beside two weight stages (MOE_EINVAL
+ * otherwise).
  * Errors: MOE_EINVAL. */
 int moe_expert_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const int32_t* idx,
                    const float* w, const int32_t* slot_of, float* y_part, void* y_bf16, int* status,
                    void* stream);
 
 /* Limits of the device-side bounded waits of moe_expert_ffn, in milliseconds:
- * a missed expert's ready flag (default 5000), the wait for the other CTAs of
- * a cluster to publish their slices of h (default 5000), a shared-memory
- * pipeline stage (default 10000).
+ * a missed expert's ready flag (default 5000), the wait for other CTAs to
+ * publish an expert's h (default 5000), a shared-memory pipeline stage
+ * (default 10000).
  * Process-wide; affects later launches.  Errors: MOE_EINVAL (non-positive). */
 int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_ms);
 
-/* Cluster size of later moe_expert_ffn launches (for tuning sweeps): 1, 2, 4, 8
- * or 16 CTAs per expert where the shapes and the GPU allow it (otherwise the
- * automatic choice); 0 = automatic (the default: the size with the least work
- * per CTA, counting the rounds in which the clusters take the experts).
- * Process-wide.  Errors: MOE_EINVAL. */
-int moe_set_ffn_cluster(int cluster);
-
 /* Launch shape moe_expert_ffn uses on this pool for T tokens (for reports):
- * CTAs per cluster, clusters launched, shared-memory weight stages per CTA,
+ * CTAs launched, shared-memory weight stages per CTA and bytes per stage,
  * dynamic shared memory per CTA in bytes.  Errors: MOE_EINVAL. */
-int moe_ffn_launch_info(moe_pool* pool, int T, int* cluster, int* clusters, int* nstage, int* smem_bytes);
+int moe_ffn_launch_info(moe_pool* pool, int T, int* ctas, int* nstage, int* stage_bytes, int* smem_bytes);
 
 /* Tracing (for profiling): when buf is a device buffer of at least 32 u64 per
  * CTA of the largest launch (32 * 296 covers every launch), each CTA of every
  * later moe_expert_ffn launch writes, at row blockIdx * 32, global-timer stamps
- * in ns: [0] start, [1] activations staged and the cluster started,
- * [2] the preceding kernel (the slot lookup) complete, [3] group table built,
- * [4] first weights landed, [5] first group's slice of h done, [6] the cluster's
- * slices published, [7] whole h gathered, [8] first group's down rows done,
- * [9] last group counted (and combined), [10] end, [11] the producer's last copy
- * issued, [16 + s] stage s of the first group landed (consumer side, s < 8),
- * [24 + s] the producer's copies of its s-th stage issued (s < 8); and counts:
- * [12] groups of the CTA, [13] CTAs per cluster, [14] rank in the cluster.
+ * in ns: [0] start, [1] activations staged, [2] the preceding kernel (the slot
+ * lookup) complete, [3] group table built, [4] first weights landed, [5] the
+ * CTA's gate/up tiles done, [6] h of its first down tile's expert complete,
+ * [7] that h in shared memory, [8] the CTA's down tiles done, [10] end,
+ * [11] the producer's last copy issued, [16 + s] the CTA's stage s landed
+ * (consumer side, s < 8), [24 + s] the producer's copies of stage s issued
+ * (s < 8); and counts: [12] gate/up tiles of the CTA, [13] its down tiles,
+ * [14] the K split of its gate/up units.
  * Unwritten entries keep their old value.  NULL turns tracing off. */
 int moe_set_ffn_trace(void* buf);
 

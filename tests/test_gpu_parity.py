@@ -239,7 +239,8 @@ def check_layer(w, lo, x, wr, b, layer, renorm=1):
     ("mxfp4", 256, 256, 16, 2, 16, 4),     # the tiny workload's shape, all resident
     ("nvfp4", 512, 256, 8, 2, 6, 3),       # misses every step, ragged T
     ("nvfp4", 768, 512, 12, 3, 12, 16),    # max tokens: pool holds one layer, misses on switch
-    ("mxfp4", 1024, 768, 10, 4, 8, 2)])
+    ("mxfp4", 1024, 768, 10, 4, 8, 2),
+    ("mxfp4", 512, 512, 16, 4, 16, 12)])   # MXFP4 past 8 tokens (two 8-column tiles)
 def test_decode_layer_small(m, fmt, H, I, E, k, S, T):
     w = small(f"d{H}", fmt, H=H, I=I, E=E, k=k, L=2)
     pool = m.Pool(H, I, E, k, 2, fmt, S, max_tokens=T)
