@@ -207,6 +207,61 @@ def ffn_roofline(torch, m, w, pool, T, x_dev, wr, bias, reps=4):
     return ms, uniq
 
 
+def resident_run(torch, m, w, pool, T, x_dev, wr, bias, reps=10):
+    """The all-resident decode of all L layers (router, resident lookup, FFN with the
+    fused combine; no host wait) captured in one CUDA graph and replayed: ms per
+    layer.  Also the per-layer host call (moe_decode_layer) on the same pool and
+    inputs for comparison."""
+    L_ = w.L
+    idx = torch.empty((T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((T, w.k), dtype=torch.float32, device="cuda")
+    slot_of = torch.empty((T, w.k), dtype=torch.int32, device="cuda")
+    y_part = torch.empty((T, w.k, w.H), dtype=torch.float32, device="cuda")
+    y = torch.empty((L_, T, w.H), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(m.route_workspace_bytes(T, w.E), dtype=torch.uint8, device="cuda")
+    wrs, bs = [wr] * L_, [bias] * L_
+
+    def run(stream):
+        m.decode_resident(pool, 0, x_dev, wrs, bs, 1, idx, wt, slot_of, y_part, y, status, ws, stream=stream)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            run(s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run(torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(20_000_000)
+    e0.record(cur)
+    for _ in range(reps):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    graph_ms = e0.elapsed_time(e1) / (reps * L_)
+    ok = int(status.item()) == 0
+    del g
+    lo = m.DecodeLayer(pool, T)
+    for l in range(L_):
+        lo(l, x_dev[l], wr, bias)
+    torch.cuda.synchronize()
+    e0.record(cur)
+    for _ in range(2):
+        for l in range(L_):
+            lo(l, x_dev[l], wr, bias)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    call_ms = e0.elapsed_time(e1) / (2 * L_)
+    return dict(graph_ms=graph_ms, call_ms=call_ms, status_ok=ok and int(lo.status.item()) == 0)
+
+
 def expert_bytes_alg(w):
     """Algorithmic HBM bytes of one expert: FP4 codes + block scales of gate, up, down."""
     bs = W.block_elems(w.fmt)
@@ -323,6 +378,46 @@ def oracle_sample(w, T, experts, budget_s=10.0, min_layers=2):
     return dict(value=T / (per_layer * w.L), unit="tokens/s", cores=1, kind="oracle",
                 sample=f"{n} (step, layer) evaluations of routing + LRU + FFN at T={T}, "
                        f"{busy:.1f} s on one host core, extrapolated to {w.L} layers")
+
+
+def oracle_sample_all_cores(w, T, experts, budget_s=10.0):
+    """The same oracle pipeline with the FFN of successive (step, layer) pairs spread
+    over every host core (one thread each; the C oracle releases the GIL): routing
+    and the LRU stay serial, as they carry state.  Timed as wall clock over the whole
+    sample; tokens/s extrapolated to all L layers."""
+    import concurrent.futures as cf
+    import oracle
+    cores = os.cpu_count() or 1
+    lru = oracle.LRU(W.n_slots(w), w.L, w.E)
+    wr = gen.router_weight(w, 0)
+    b = gen.router_bias(w, 0)
+    xs = []
+    n = 0
+    # size the sample from one single-thread layer, so the wall time stays near budget_s
+    x = gen.activations(w, 0, 0, T)
+    ta = time.perf_counter()
+    idx, wt, _ = oracle.route(x, wr, b, w.k, 1)
+    oracle.moe_decode(w.fmt, w.H, w.I, w.E, x, idx, wt, {e: experts[e] for e in set(idx.ravel().tolist())})
+    one = time.perf_counter() - ta
+    n_items = max(cores, int(budget_s * cores / max(one, 1e-6)))
+    n_items = min(n_items, 64 * cores)
+    for i in range(n_items):
+        s_, l = divmod(i, w.L)
+        xs.append((l, gen.activations(w, l, s_, T)))
+    t0 = time.perf_counter()
+    jobs = []
+    with cf.ThreadPoolExecutor(cores) as ex:
+        for l, x in xs:
+            idx, wt, _ = oracle.route(x, wr, b, w.k, 1)
+            lru.step(l, idx)
+            sub = {e: experts[e] for e in set(idx.ravel().tolist())}
+            jobs.append(ex.submit(oracle.moe_decode, w.fmt, w.H, w.I, w.E, x, idx, wt, sub))
+        for j in jobs:
+            j.result()
+    wall = time.perf_counter() - t0
+    return dict(value=T * n_items / (wall * w.L), unit="tokens/s", cores=cores, kind="oracle",
+                sample=f"{n_items} (step, layer) evaluations at T={T}, FFN on {cores} threads, "
+                       f"{wall:.1f} s wall, extrapolated to {w.L} layers")
 
 
 def ffn_only(args, w, T):
@@ -450,30 +545,57 @@ def offload_mode(args):
             v = W.stress_variant(zs, pf)
             runs.append((v.name, v, W.n_slots(v), zs, W.STRESS_284B.steps))
     for name, v, slots, zs, steps in runs:
-        bias = [torch.from_numpy(gen.router_bias(v, l, zs)).cuda() for l in range(w.L)]
-        pool.reset(slots)
-        r = decode_run(torch, m, w, pool, 1, xs_dev, wr, bias, steps, args.warmup, events=True,
-                       overlap=not args.no_overlap)
-        st = r["stats"]
-        copy_ms = sum(t for t, _ in r["copy"])
-        t_comp = t_layer * w.L * steps
-        m_layer = st["misses"] / (steps * w.L)
-        q = {f"{bp}/{bh}": dict(zip(("q_gpu", "q_cpu", "ratio"), m.qstar_split(int(round(m_layer)), bp, bh)))
-             for bp, bh in W.QSTAR_MACHINES}
-        line = {"mode": "offload", "run": name, "zipf_s": zs, "slots": slots,
-                "slot_frac": round(slots / (w.L * w.E), 4), "steps": steps, "warmup": args.warmup,
-                "tokens_per_s": round(steps / (r["ms"] * 1e-3), 3), "ms_per_step": round(r["ms"] / steps, 4),
-                "hit_rate": round(st["hits"] / max(1, st["unique"]), 4),
-                "misses_per_layer": round(m_layer, 3),
-                "h2d_gbs": round(st["h2d_bytes"] / (copy_ms * 1e-3) / 1e9, 2) if copy_ms > 0 else None,
-                "h2d_bytes_per_step": st["h2d_bytes"] // steps,
-                "t_wall_ms": round(r["ms"], 2), "t_copy_ms": round(copy_ms, 2), "t_comp_ms": round(t_comp, 2),
-                "overlap_efficiency": overlap_efficiency(r["ms"], copy_ms, t_comp),
-                "qstar_per_layer": q, "status": r["status"],
-                "host_store": f"{HL} distinct layer weight sets for {w.L} layer positions",
-                "store_load_s": round(load_s, 1)}
+        line = offload_run(torch, m, w, pool, v, slots, zs, steps, args.warmup, xs_dev, wr, t_layer,
+                           not args.no_overlap)
+        line.update({"mode": "offload", "run": name,
+                     "host_store": f"{HL} distinct layer weight sets for {w.L} layer positions",
+                     "store_load_s": round(load_s, 1)})
         print(json.dumps(line), flush=True)
     pool.close()
+
+
+def offload_run(torch, m, w, pool, v, slots, zs, steps, warmup, xs_dev, wr, t_layer, overlap):
+    """One offload run on `slots` slots with variant v's routing bias: tokens/s, hit
+    rate, H2D GB/s, overlap efficiency and the q* split for the pages' machines."""
+    bias = [torch.from_numpy(gen.router_bias(v, l, zs)).cuda() for l in range(w.L)]
+    pool.reset(slots)
+    r = decode_run(torch, m, w, pool, 1, xs_dev, wr, bias, steps, warmup, events=True, overlap=overlap)
+    st = r["stats"]
+    copy_ms = sum(t for t, _ in r["copy"])
+    t_comp = t_layer * w.L * steps
+    m_layer = st["misses"] / (steps * w.L)
+    q = {f"{bp}/{bh}": dict(zip(("q_gpu", "q_cpu", "ratio"), m.qstar_split(int(round(m_layer)), bp, bh)))
+         for bp, bh in W.QSTAR_MACHINES}
+    return {"zipf_s": zs, "slots": slots, "slot_frac": round(slots / (w.L * w.E), 4), "steps": steps,
+            "warmup": warmup, "tokens_per_s": round(steps / (r["ms"] * 1e-3), 3),
+            "ms_per_step": round(r["ms"] / steps, 4),
+            "hit_rate": round(st["hits"] / max(1, st["unique"]), 4),
+            "misses_per_layer": round(m_layer, 3),
+            "h2d_gbs": round(st["h2d_bytes"] / (copy_ms * 1e-3) / 1e9, 2) if copy_ms > 0 else None,
+            "h2d_bytes_per_step": st["h2d_bytes"] // steps,
+            "t_wall_ms": round(r["ms"], 2), "t_copy_ms": round(copy_ms, 2), "t_comp_ms": round(t_comp, 2),
+            "overlap_efficiency": overlap_efficiency(r["ms"], copy_ms, t_comp),
+            "qstar_per_layer": q, "status": r["status"]}
+
+
+def offload_summary(torch, m, overlap, steps=8, warmup=12):
+    """decode_284b on its 2570-slot (32 GiB) pool for the default line, bounded in
+    time: one host layer of generated experts serves all 40 layer positions (the LRU
+    still keys every (layer, expert)); warm-up steps fill the pool first."""
+    w = W.DECODE_284B
+    pool = m.Pool(w.H, w.I, w.E, w.k, w.L, w.fmt, W.n_slots(w), max_tokens=1, host_layers=1)
+    t0 = time.perf_counter()
+    load_mxfp4_store(m, w, pool, 1)
+    load_s = time.perf_counter() - t0
+    xs = np.stack([np.stack([gen.activations(w, l, s, 1) for l in range(w.L)]) for s in range(warmup + steps)])
+    xs_dev = torch.from_numpy(xs.view(np.int16)).cuda().view(torch.bfloat16)
+    wr = [torch.from_numpy(gen.router_weight(w, l).view(np.int16)).cuda().view(torch.bfloat16) for l in range(w.L)]
+    t_layer = resident_layer_ms(torch, m, w, pool, xs_dev, wr, [None] * w.L)
+    line = offload_run(torch, m, w, pool, w, W.n_slots(w), w.zipf_s, steps, warmup, xs_dev, wr, t_layer, overlap)
+    pool.close()
+    line.update({"workload": w.name, "host_store": "1 layer weight set for 40 layer positions",
+                 "store_load_s": round(load_s, 1), "resident_layer_ms": round(t_layer, 4)})
+    return line
 
 
 # ---------------------------------------------------------------------- main
@@ -558,7 +680,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=4)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batch", type=int, default=1, help="decode tokens per step (1, 4 or 8)")
-    ap.add_argument("--all-batches", action="store_true", help="also time batches 4 and 8")
+    ap.add_argument("--no-offload", action="store_true",
+                    help="skip the decode_284b offload run of the default line")
     ap.add_argument("--oracle-budget", type=float, default=10.0)
     ap.add_argument("--mode", default="decode", choices=["decode", "ffn", "prefill", "offload"],
                     help="ffn: only the decode FFN kernel on a small all-resident pool "
@@ -642,7 +765,7 @@ def main():
     host_layers = w.L if world == 1 else 12
     pool = make_pool(m, w, W.n_slots(w), 8, host_layers, experts)
     res = {}
-    batches = [T] + ([b for b in (1, 4, 8) if b != T] if args.all_batches else [])
+    batches = [T] + [b for b in W.DECODE_35B.batches if b != T]
     sampler = ClockSampler(local)
     for b in batches:
         xd = dev_x(b)
@@ -669,22 +792,30 @@ def main():
     pool_block_bytes = pool.block_bytes
     pool.close()
 
-    # all-resident pool: the FFN kernel's own HBM roofline on the same layers
+    # all-resident pool: the FFN kernel's own HBM roofline on the same layers, per batch
     rpool = make_pool(m, w, w.L * w.E, 8, 1, experts)
     preload(torch, m, rpool, w)
-    xd = dev_x(T)
-    ffn_ms, ffn_u = ffn_roofline(torch, m, w, rpool, T, xd[0], wr, bias)
+    roof = {}
+    for b in batches:
+        xd = dev_x(b)
+        b_ms, b_u = ffn_roofline(torch, m, w, rpool, b, xd[0], wr, bias)
+        b_alg = sum(ffn_alg_bytes(w, b, u) for u in b_u) / len(b_u)
+        roof[b] = dict(ms=b_ms, alg=b_alg, gbs=b_alg / (b_ms * 1e-3) / 1e9,
+                       uniq=sum(b_u) / len(b_u))
+        if b == T:
+            resid = resident_run(torch, m, w, rpool, b, xd[0], wr, bias)
+        del xd
     rpool.close()
-    per_exp = expert_bytes_alg(w)
-    alg_bytes = [ffn_alg_bytes(w, T, u) for u in ffn_u]
-    alg_avg = sum(alg_bytes) / len(alg_bytes)
-    achieved = alg_avg / (ffn_ms * 1e-3) / 1e9
+    ffn_ms, alg_avg, achieved = roof[T]["ms"], roof[T]["alg"], roof[T]["gbs"]
+
+    # decode_284b through the offload path (bounded), for the compact offload object
+    off = offload_summary(torch, m, not args.no_overlap) if world == 1 and not args.no_offload else None
 
     # prefill of the same layer: a 2048-token prompt, all experts resident
     wp = W.PREFILL_35B
     pr = prefill_run(torch, m, wp, 2048, experts)
     pfl = prefill_flops(wp, 2048)
-    _, bf16_peak, _ = peaks()
+    _, bf16_peak, bf16_kind = peaks()
     fp4_peak = bf16_peak * FP4_PER_BF16
 
     # reduce over ranks: max time, summed tokens
@@ -702,7 +833,10 @@ def main():
     qstar_rt = qstar_runtime(m, r["copy"], pool_block_bytes, st["misses"] / max(1, args.steps * w.L))
 
     if rank == 0:
-        cb = oracle_sample(w, T, experts, budget_s=args.oracle_budget) if world == 1 else None
+        cb = None
+        if world == 1:
+            cb = oracle_sample(w, T, experts, budget_s=args.oracle_budget)
+            cb["all_cores"] = oracle_sample_all_cores(w, T, experts, budget_s=args.oracle_budget)
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
@@ -717,21 +851,36 @@ def main():
                          "alg_bytes_per_launch_avg": int(alg_avg)},
             "e2e": {"value": round(replica_value(T * args.steps, world, e2e_ms), 3), "unit": "tokens/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
-            "gpu_launches": 4 * w.L * args.steps,
+            "gpu_launches": 3 * w.L * args.steps,   # router, slot lookup, FFN (combine fused) per layer
             "clocks": clocks,
             "h2d_gbs": round(h2d_gbs, 2) if h2d_gbs else None,
             "qstar_runtime": qstar_rt,
             "h2d_bytes_per_step": st["h2d_bytes"] // args.steps,
             "hit_rate": round(st["hits"] / max(1, st["unique"]), 4),
             "misses_per_layer": round(st["misses"] / (args.steps * w.L), 3),
-            "batches": {str(b): round(b * args.steps / (res[b]["ms"] * 1e-3), 3) for b in res},
+            "batches": {str(b): {"tokens_per_s": round(b * args.steps / (res[b]["ms"] * 1e-3), 3),
+                                 "hit_rate": round(res[b]["stats"]["hits"] / max(1, res[b]["stats"]["unique"]), 4),
+                                 "roofline": {"bound": "hbm", "achieved": round(roof[b]["gbs"], 1),
+                                              "peak": hbm_peak, "unit": "GB/s",
+                                              "frac": round(roof[b]["gbs"] / hbm_peak, 4),
+                                              "launch_ms_avg": round(roof[b]["ms"], 5),
+                                              "alg_bytes_per_launch_avg": int(roof[b]["alg"]),
+                                              "unique_experts_avg": round(roof[b]["uniq"], 2)}}
+                        for b in res},
+            "offload": off,
+            "resident_decode": {"workload": w.name, "batch": T, "layers": w.L, "pool": "all L*E experts resident",
+                                "graph_ms_per_layer": round(resid["graph_ms"], 5),
+                                "ffn_ms_per_layer": round(ffn_ms, 5),
+                                "overhead_us_per_layer": round((resid["graph_ms"] - ffn_ms) * 1e3, 2),
+                                "per_layer_call_ms": round(resid["call_ms"], 5),
+                                "status_ok": resid["status_ok"]},
             "status": r["status"],
             "prefill": {"workload": wp.name, "tokens": 2048, "ffn_ms": round(pr["ffn_ms"], 4),
                         "combine_ms": round(pr["combine_ms"], 4), "flops": pfl,
                         "tflops": round(pfl / (pr["ffn_ms"] * 1e-3) / 1e12, 1),
                         "peak_tflops": fp4_peak,
                         "frac": round(pfl / (pr["ffn_ms"] * 1e-3) / 1e12 / fp4_peak, 4),
-                        "peak_source": "measured bf16 x 4 (nominal FP4:BF16 ratio)",
+                        "peak_source": f"{bf16_kind} bf16 x 4 (nominal FP4:BF16 ratio)",
                         "status_ok": pr["status_ok"]},
         }
         if cb is not None:

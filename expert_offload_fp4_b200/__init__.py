@@ -4,8 +4,8 @@ miss streaming, FP4 SwiGLU expert FFN, router-weighted combine, and the q*
 bandwidth split.  The work is in libmoe_fp4.so (include/moe_fp4.h); this package
 is its Python binding."""
 from . import _lib  # noqa: F401
-from .api import (BandwidthEstimate, Lookup, Pool, combine, decode_layer, dequant_slot, expert_ffn,  # noqa: F401
-                  ffn_launch_info, nvfp4_gemm,
+from .api import (BandwidthEstimate, Lookup, Pool, combine, decode_layer, decode_resident,  # noqa: F401
+                  dequant_slot, expert_ffn, ffn_launch_info, nvfp4_gemm,
                   nvfp4_quantize, prefill_ffn, prefill_workspace_bytes, qstar_split,
                   route, route_noalloc, route_workspace_bytes, set_wait_limits, slot_lookup,
                   slot_lookup_launch, slot_lookup_result, stream_misses)

@@ -17,6 +17,7 @@ MOE_MXFP4, MOE_NVFP4 = 0, 1
 MOE_COPY_SM, MOE_COPY_DMA = 0, 1
 MOE_BW_PCIE, MOE_BW_HOST = 0, 1
 STATUS_READY_TIMEOUT, STATUS_DEP_TIMEOUT, STATUS_BAD_SLOT, STATUS_BAD_EXPERT, STATUS_PIPE_TIMEOUT = 1, 2, 4, 8, 16
+STATUS_NOT_RESIDENT = 32
 
 
 class MoeConfig(C.Structure):
@@ -84,6 +85,8 @@ SIGNATURES = {
     "moe_combine": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_decode_layer": (i32, [vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,
                                C.POINTER(LookupResult), vp, vp, i32, vp, vp]),
+    "moe_decode_resident": (i32, [vp, i32, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,
+                                  vp]),
     "qstar_split": (i32, [i32, f64, f64, C.POINTER(i32), C.POINTER(i32), C.POINTER(f64)]),
     "moe_bw_init": (i32, [C.POINTER(BwEstimate), f64, f64, f64]),
     "moe_bw_observe": (i32, [C.POINTER(BwEstimate), i32, f64, f64]),

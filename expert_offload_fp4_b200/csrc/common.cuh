@@ -36,6 +36,9 @@ constexpr int kMaxK = 32;            // experts per token
 constexpr int kMaxDecodeT = 16;      // tokens of one decode FFN call
 constexpr int kMaxDecodePairs = 128; // (token, rank) pairs of one decode FFN call
 constexpr int kMaxSlots = 1 << 20;
+// A slot's ready word shows (ticket | kTicketPartA) once the gate and up tensors of
+// its copy have landed, then the ticket itself once the whole block has.
+constexpr uint32_t kTicketPartA = 0x80000000u;
 
 // Per-call output of the lookup kernel, in mapped pinned host memory.
 struct LookupOut {
@@ -62,6 +65,8 @@ int preload_gemm_kernels();
 int preload_prefill_kernels();
 int preload_pull_kernels();
 cudaError_t launch_pull(const uint8_t* src_d, uint8_t* dst, size_t bytes, int num_sms, cudaStream_t s);
+int launch_lookup(moe_pool* p, int layer, const int32_t* idx, int T, int k, int32_t* slot_of, cudaStream_t s,
+                  int resident, int* status);
 
 }  // namespace moe
 

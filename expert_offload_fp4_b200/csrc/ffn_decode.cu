@@ -50,7 +50,8 @@ constexpr int kFfnMaxRegs = 96;
 constexpr int kSeg = 128;                    // K elements per segment (64 code bytes)
 
 struct Group {
-    int expert, slot, M, ready;
+    int expert, slot, M;
+    int ready_a, ready_b;      // the slot showed gate/up (a) or the whole block (b) at table time
     unsigned need;
     float ts[3];
     float wt[kMaxDecodeT];     // routing weight of each member (token, rank)
@@ -177,12 +178,14 @@ __device__ __forceinline__ unsigned ld_acquire_gpu_u32(const unsigned int* p) {
     return v;
 }
 
-__device__ __forceinline__ bool wait_ready(const uint32_t* ready, uint32_t want, unsigned long long limit_ns,
-                                           volatile unsigned int* abort_flag) {
-    if (ld_acquire_gpu_u32(ready) == want) return true;
+// Bounded wait until (*ready & mask) == want: mask ~kTicketPartA for the gate/up
+// part of a copy, all ones for the whole block.
+__device__ __forceinline__ bool wait_ready(const uint32_t* ready, uint32_t want, uint32_t mask,
+                                           unsigned long long limit_ns, volatile unsigned int* abort_flag) {
+    if ((ld_acquire_gpu_u32(ready) & mask) == want) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
-        if (ld_acquire_gpu_u32(ready) == want) return true;
+        if ((ld_acquire_gpu_u32(ready) & mask) == want) return true;
         if (*abort_flag) return false;
         if (globaltimer() - t0 > limit_ns) return false;
         __nanosleep(64);
@@ -449,7 +452,7 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
         e_s[tid] = bad ? -1 : e;
         s_s[tid] = sl;
         need_s[tid] = nd;
-        rdy_s[tid] = (rd == nd);
+        rdy_s[tid] = ((rd & ~kTicketPartA) == nd) | ((rd == nd) << 1);
         gm_s[tid] = 0;
         if (bad && blockIdx.x == 0) atomicOr(a.status, bad);
     }
@@ -489,7 +492,8 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
         G.expert = e;
         G.slot = s_s[ld];
         G.M = gm_s[ld];
-        G.ready = rdy_s[ld];
+        G.ready_a = rdy_s[ld] & 1;
+        G.ready_b = rdy_s[ld] >> 1;
         G.need = need_s[ld];
         G.ts[0] = ts_row[3 * e];
         G.ts[1] = ts_row[3 * e + 1];
@@ -522,22 +526,26 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
 
     if (warp == kNC) {
         // ---------------------------------------------------------------- producer
-        int st = 0, issued = 0, lastg = -1;
+        int st = 0, issued = 0, lastg = -1, lastpart = 0;
         uint32_t round = 0;
         const uint8_t* blk = nullptr;
-        // first use of a group's slot: a slot that showed its ticket when the table
-        // was built was acquired then (and the CTA barrier since orders it); for a
-        // pending one, wait (bounded) for the ticket and acquire it here.  Then the
-        // bulk (async proxy) reads are ordered after the acquire.
+        // first use of a group's slot for gate/up (part 0) or down (part 1): a slot
+        // that showed that part when the table was built was acquired then (and
+        // the CTA barrier since orders it); for a pending one, wait (bounded) for
+        // the part's ticket and acquire it here.  Then the bulk (async proxy)
+        // reads are ordered after the acquire.
         fence_proxy_async_global();
         if (trace && lane == 0) trace[9] = globaltimer();
-        auto use_group = [&](int g) {
-            if (g == lastg) return;
+        auto use_group = [&](int g, int part) {
+            if (g == lastg && part == lastpart) return;
             lastg = g;
+            lastpart = part;
             const Group& G = groups[g];
-            if (!G.ready) {
+            if (!(part ? G.ready_b : G.ready_a)) {
                 bool ok = true;
-                if (lane == 0) ok = wait_ready(a.ready + G.slot, G.need, a.ready_ns, abort_flag);
+                if (lane == 0)
+                    ok = wait_ready(a.ready + G.slot, G.need, part ? 0xFFFFFFFFu : ~kTicketPartA, a.ready_ns,
+                                    abort_flag);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok && lane == 0) {
                     atomicOr(a.status, MOE_STATUS_READY_TIMEOUT);
@@ -571,7 +579,7 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
         // A item: 16 rows of gate and the same rows of up, codes then scales
         for (int i = a0; i < a1; i++) {
             const int g = i / nTA, t = i - g * nTA;
-            use_group(g);
+            use_group(g, 0);
             uint8_t* dst = take_slot(2 * CA + 2 * 16 * SA);
             const unsigned long long r0 = (unsigned long long)t * 16;
             if (lane == 0) bulk_g2s(dst, blk + a.off[0] + r0 * (H / 2), CA, &full[st]);
@@ -585,7 +593,7 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
             int g, r, nt;
             bstage(i, g, r, nt);
             i += nt;
-            use_group(g);
+            use_group(g, 1);
             const uint32_t cb = (uint32_t)nt * 16 * (I / 2), sbb = (uint32_t)nt * 16 * SB;
             uint8_t* dst = take_slot(cb + sbb);
             const unsigned long long r0 = (unsigned long long)r * 16;

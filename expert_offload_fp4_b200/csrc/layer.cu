@@ -53,3 +53,31 @@ extern "C" int moe_decode_layer(moe_pool* p, int layer, const void* x_bf16, int 
     if (rc2) return rc2;
     return copies();
 }
+
+// All-resident decode of consecutive layers (post.smzdm.com/p/aomxznrn,
+// "FreeToken干的事": decode is scheduled on its own, bandwidth-bound path): per
+// layer the router, the lookup in its resident form and the FFN with the fused
+// combine, chained by programmatic stream serialisation with no host wait in
+// between, so a caller may capture the whole sequence in one CUDA graph.
+extern "C" int moe_decode_resident(moe_pool* p, int layer0, int n_layers, const void* x_bf16, int T,
+                                   const void* const* wr_bf16, const float* const* bias, int renormalize,
+                                   int32_t* idx, float* w, int32_t* slot_of, float* y_part, void* y_bf16,
+                                   int* status, void* route_ws, size_t route_ws_bytes, void* stream) {
+    if (!p || !x_bf16 || !wr_bf16 || !y_bf16 || !status) return fail(MOE_EINVAL, "null argument");
+    const moe_config& c = p->cfg;
+    if (n_layers <= 0 || layer0 < 0 || layer0 + n_layers > c.L) return fail(MOE_EBOUNDS, "layers outside the pool");
+    if (T <= 0 || T > c.max_tokens) return fail(MOE_EINVAL, "T must be in [1, max_tokens]");
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t xl = (size_t)T * c.H * 2;
+    for (int i = 0; i < n_layers; i++) {
+        if (!wr_bf16[i]) return fail(MOE_EINVAL, "null router weight");
+        const uint8_t* x = (const uint8_t*)x_bf16 + i * xl;
+        uint8_t* y = (uint8_t*)y_bf16 + i * xl;
+        int rc = moe_route(x, wr_bf16[i], bias ? bias[i] : nullptr, T, c.H, c.E, c.k, renormalize, idx, w, route_ws,
+                           route_ws_bytes, stream);
+        if (rc) return rc;
+        if ((rc = launch_lookup(p, layer0 + i, idx, T, c.k, slot_of, s, 1, status))) return rc;
+        if ((rc = moe_expert_ffn(p, layer0 + i, x, T, idx, w, slot_of, y_part, y, status, stream))) return rc;
+    }
+    return MOE_OK;
+}

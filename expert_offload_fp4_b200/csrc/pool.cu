@@ -360,6 +360,8 @@ extern "C" int moe_pool_slot_ptr(moe_pool* p, int slot, void** ptr, size_t* byte
 
 typedef CUresult (*write_value32_fn)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
 
+constexpr size_t kSplitBytes = size_t(8) << 20;   // blocks at least this large are copied in two parts
+
 extern "C" int moe_stream_misses(moe_pool* p, int layer, const moe_miss* miss_h, int n_miss,
                                  void* copy_stream) {
     if (!p) return fail(MOE_EINVAL, "null pool");
@@ -377,17 +379,29 @@ extern "C" int moe_stream_misses(moe_pool* p, int layer, const moe_miss* miss_h,
             return fail(MOE_ESTATE, "missed expert was never loaded into the host store");
     }
     auto wv = (write_value32_fn)p->write_value32;
+    // large blocks go in two parts: gate and up (codes and scales, the block's
+    // first bytes), published as ticket | kTicketPartA, then down, published as
+    // the ticket; the FFN starts a missed expert's gate/up rows while its down
+    // rows are still crossing.  A block under kSplitBytes goes in one copy: the
+    // second copy's fixed cost outweighs the overlap there.
+    const size_t part_a = p->lay.off[4];
+    const int parts = p->lay.bytes >= kSplitBytes ? 2 : 1;
     for (int i = 0; i < n_miss; i++) {
         const moe_miss& m = miss_h[i];
         const uint8_t* src = p->host + (size_t(hl) * c.E + m.expert) * p->lay.bytes;
         uint8_t* dst = p->slots + size_t(m.slot) * p->lay.bytes;
-        if (p->copy_mode == MOE_COPY_DMA) {
-            MOE_CUDA_TRY(cudaMemcpyAsync(dst, src, p->lay.bytes, cudaMemcpyHostToDevice, s));
-        } else {
-            MOE_CUDA_TRY(launch_pull(p->host_d + (src - p->host), dst, p->lay.bytes, p->num_sms, s));
+        for (int part = 2 - parts; part < 2; part++) {
+            const size_t o = part && parts == 2 ? part_a : 0;
+            const size_t n = parts == 1 ? p->lay.bytes : part ? p->lay.bytes - part_a : part_a;
+            if (p->copy_mode == MOE_COPY_DMA) {
+                MOE_CUDA_TRY(cudaMemcpyAsync(dst + o, src + o, n, cudaMemcpyHostToDevice, s));
+            } else {
+                MOE_CUDA_TRY(launch_pull(p->host_d + (src - p->host) + o, dst + o, n, p->num_sms, s));
+            }
+            const uint32_t v = part ? m.ticket : (m.ticket | kTicketPartA);
+            CUresult r = wv((CUstream)s, (CUdeviceptr)(p->ready + m.slot), v, 0);
+            if (r != CUDA_SUCCESS) return fail(MOE_ECUDA, "cuStreamWriteValue32 failed");
         }
-        CUresult r = wv((CUstream)s, (CUdeviceptr)(p->ready + m.slot), m.ticket, 0);
-        if (r != CUDA_SUCCESS) return fail(MOE_ECUDA, "cuStreamWriteValue32 failed");
         p->stats.h2d_bytes += (long long)p->lay.bytes;
         p->stats.h2d_copies += 1;
     }

@@ -66,7 +66,8 @@ enum {
     MOE_STATUS_DEP_TIMEOUT = 2,    /* waited too long for an expert's h (other CTAs) */
     MOE_STATUS_BAD_SLOT = 4,       /* slot index outside the pool */
     MOE_STATUS_BAD_EXPERT = 8,     /* expert index outside [0, E) */
-    MOE_STATUS_PIPE_TIMEOUT = 16   /* a shared-memory pipeline wait gave up */
+    MOE_STATUS_PIPE_TIMEOUT = 16,  /* a shared-memory pipeline wait gave up */
+    MOE_STATUS_NOT_RESIDENT = 32   /* moe_decode_resident: an expert was not resident */
 };
 
 typedef struct {
@@ -224,11 +225,17 @@ int moe_slot_lookup_result(moe_pool* pool, moe_lookup_result* res);
 
 /* Miss streaming ("游戏电脑如何跑动2840亿参数大模型": prefetch with a double
  * buffer, copies in the background while computing).  For each miss, in order,
- * one cudaMemcpyAsync of the expert's pinned host block into its slot on
- * copy_stream, then a stream write of the ticket into the slot's ready flag.
- * moe_expert_ffn starts at once on another stream; its CTAs on missed experts
- * wait (bounded) for the flag, so the copy of miss j+1 overlaps compute on the
- * hits and on miss j.  When the FFN is enqueued before the misses are streamed
+ * the expert's pinned host block is copied into its slot on copy_stream (one
+ * cudaMemcpyAsync per part, or a copy kernel in MOE_COPY_SM mode).  A block of
+ * 8 MiB or more goes in two parts: first the gate and up tensors (codes and
+ * scales, the block's leading bytes), then a stream write of
+ * ticket | 0x80000000 into the slot's ready word; then the down tensors, then
+ * a stream write of the ticket itself.  A smaller block goes in one copy
+ * followed by the ticket.  moe_expert_ffn starts at
+ * once on another stream; its gate/up work on a missed expert waits (bounded)
+ * for the first value and its down work for the second, so the copy of miss j+1
+ * overlaps compute on the hits and on miss j, and a miss's gate/up rows are
+ * consumed while its down rows are still crossing.  When the FFN is enqueued before the misses are streamed
  * (moe_slot_lookup_launch, moe_expert_ffn, moe_slot_lookup_result, then this
  * call), the host must not wait for the device in between (a synchronize, a
  * blocking allocation, a first launch of a lazily loaded kernel): the FFN would
@@ -367,6 +374,28 @@ int moe_decode_layer(moe_pool* pool, int layer, const void* x_bf16, int T, const
                      float* y_part, void* y_bf16, int* status, void* route_ws,
                      size_t route_ws_bytes, moe_lookup_result* res, void* copy_start,
                      void* copy_end, int overlap, void* stream, void* copy_stream);
+
+/* All-resident decode of layers layer0 .. layer0+n_layers-1 (post.smzdm.com/p/
+ * aomxznrn, "FreeToken干的事": decode runs on its own bandwidth-bound path): per
+ * layer moe_route, the slot lookup and moe_expert_ffn with the combine fused in,
+ * on `stream`, with no host wait anywhere, so the call may be captured into a
+ * CUDA graph and replayed.  Every expert the layers touch must already be
+ * resident (for instance a pool with n_slots >= L * E after one pass of
+ * moe_decode_layer): the lookup only refreshes the LRU clocks of its hits; it
+ * never evicts, streams or writes the host record.  An expert that is not
+ * resident leaves the pool untouched, sets MOE_STATUS_NOT_RESIDENT (and
+ * MOE_STATUS_BAD_SLOT from the FFN) in *status, and that layer's output is not
+ * valid.  x_bf16: [n_layers, T, H] (device); y_bf16: [n_layers, T, H];
+ * wr_bf16, bias: host arrays of n_layers device pointers ([E, H] bf16 router
+ * weights; [E] fp32 bias or NULL; bias itself may be NULL); idx, w, slot_of
+ * ([T, k]), y_part ([T, k, H] fp32), route_ws and status as for
+ * moe_decode_layer, reused by every layer in stream order.  No lookup may be
+ * outstanding on the pool while the graph runs.  Errors: MOE_EINVAL,
+ * MOE_EBOUNDS, and those of the three calls. */
+int moe_decode_resident(moe_pool* pool, int layer0, int n_layers, const void* x_bf16, int T,
+                        const void* const* wr_bf16, const float* const* bias, int renormalize,
+                        int32_t* idx, float* w, int32_t* slot_of, float* y_part, void* y_bf16,
+                        int* status, void* route_ws, size_t route_ws_bytes, void* stream);
 
 /* q* split (post.smzdm.com/p/a825qpgl section 二: q* = m*B_p/B_h; "跑不快大模型，
  * 先别急着怪显卡" section 二: pull : compute = pcie_bw : (cpu_bw - pcie_bw)).
