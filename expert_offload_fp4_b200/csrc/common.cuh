@@ -65,8 +65,10 @@ int preload_gemm_kernels();
 int preload_prefill_kernels();
 int preload_pull_kernels();
 cudaError_t launch_pull(const uint8_t* src_d, uint8_t* dst, size_t bytes, int num_sms, cudaStream_t s);
-int launch_lookup(moe_pool* p, int layer, const int32_t* idx, int T, int k, int32_t* slot_of, cudaStream_t s,
-                  int resident, int* status);
+// The decode FFN; resident != 0 takes the slots from the pool's key table and
+// applies the slot lookup's LRU touch itself (no lookup kernel before it).
+int expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx, const float* w,
+               const int32_t* slot_of, float* y_part, void* y_bf16, int* status, void* stream, int resident);
 
 }  // namespace moe
 

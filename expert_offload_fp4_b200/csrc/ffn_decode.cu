@@ -63,7 +63,7 @@ struct FfnArgs {
     const uint16_t* x;
     const int32_t* idx;
     const float* w;
-    const int32_t* slot_of;
+    int32_t* slot_of;          // read; written by CTA 0 in resident mode
     float* y_part;
     uint16_t* y;               // bf16 output [T, H] (the fused combine), or null
     int* status;
@@ -74,6 +74,12 @@ struct FfnArgs {
     const uint32_t* need;
     const uint32_t* ready;
     float* hbuf;               // [T * k][I] h of each (token, rank), fp32
+    // resident mode (no lookup kernel before this one): slots come from key_slot;
+    // CTA 0 touches the hits' LRU clocks the way the lookup does and writes slot_of
+    const int32_t* key_slot;
+    unsigned long long* slot_clock;
+    unsigned long long* clock;
+    int resident;
     unsigned int* ctr;         // [H/16] row tiles, [kMaxDecodePairs] groups, [kMaxDecodePairs] pair maxima,
                                // abort flag, done count
     int T, k, H, I, E, S, layer;
@@ -440,10 +446,15 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     const int n = T * a.k;
     if (tid == 0) s_misc[0] = 0;
     if (tid < n) {
-        const int e = a.idx[tid], sl = a.slot_of[tid];
+        const int e = a.idx[tid];
         int bad = 0;
         if (e < 0 || e >= a.E) bad |= MOE_STATUS_BAD_EXPERT;
+        int sl = -1;
+        if (!a.resident) sl = a.slot_of[tid];
+        else if (!bad) sl = a.key_slot[(size_t)a.layer * a.E + e];
+        if (a.resident && !bad && sl < 0) bad |= MOE_STATUS_NOT_RESIDENT;
         if (sl < 0 || sl >= a.S) bad |= MOE_STATUS_BAD_SLOT;
+        if (a.resident && blockIdx.x == 0) a.slot_of[tid] = sl;
         uint32_t nd = 0u, rd = 1u;
         if (!bad) {
             nd = a.need[sl];
@@ -483,9 +494,16 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     const int nl = s_misc[0];
     if (tid < nl) {
         const unsigned long long key = lkey_s[tid];
-        int rank = 0;
+        int rank = 0, erank = 0;
 #pragma unroll 8
-        for (int j = 0; j < nl; j++) rank += lkey_s[j] < key;
+        for (int j = 0; j < nl; j++) {
+            rank += lkey_s[j] < key;
+            erank += (unsigned)lkey_s[j] < (unsigned)key;
+        }
+        if (a.resident && blockIdx.x == 0) {
+            // the lookup's touch of the hits: ascending expert id, clock = G0 + 1 + rank
+            a.slot_clock[s_s[lpos_s[tid]]] = *a.clock + 1 + erank;
+        }
         const int ld = lpos_s[tid], e = e_s[ld];
         grank_s[ld] = rank;
         Group& G = groups[rank];
@@ -508,6 +526,7 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     }
     __syncthreads();
     const int ng = s_misc[0];
+    if (a.resident && blockIdx.x == 0 && tid == 0) *a.clock += (unsigned long long)ng;
     if (trace && tid == 0) trace[3] = globaltimer();
 
     // ---- this CTA's work: A items [a0, a1) and B tiles [b0, b1) of the call's
@@ -1102,9 +1121,10 @@ extern "C" int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_m
     return MOE_OK;
 }
 
-extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx,
-                              const float* w, const int32_t* slot_of, float* y_part, void* y_bf16, int* status,
-                              void* stream) {
+namespace moe {
+
+int expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx, const float* w,
+               const int32_t* slot_of, float* y_part, void* y_bf16, int* status, void* stream, int resident) {
     if (!p || !x_bf16 || !idx || !w || !slot_of || !y_part || !status) return fail(MOE_EINVAL, "null argument");
     const moe_config& c = p->cfg;
     if (layer < 0 || layer >= c.L) return fail(MOE_EBOUNDS, "layer outside the pool");
@@ -1115,7 +1135,7 @@ extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T,
     a.x = (const uint16_t*)x_bf16;
     a.idx = idx;
     a.w = w;
-    a.slot_of = slot_of;
+    a.slot_of = const_cast<int32_t*>(slot_of);   // written only in resident mode, whose caller owns it
     a.y_part = y_part;
     a.y = (uint16_t*)y_bf16;
     a.status = status;
@@ -1127,6 +1147,10 @@ extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T,
     a.ready = p->ready;
     a.ctr = p->ctr;
     a.hbuf = p->hbuf;
+    a.resident = resident;
+    a.key_slot = p->key_slot;
+    a.slot_clock = p->slot_clock;
+    a.clock = p->clock;
     a.T = T;
     a.k = c.k;
     a.H = c.H;
@@ -1141,6 +1165,14 @@ extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T,
     cudaStream_t s = (cudaStream_t)stream;
     if (c.fmt == MOE_NVFP4) return T <= 8 ? launch_ffn<MOE_NVFP4, 1>(p, a, s) : launch_ffn<MOE_NVFP4, 2>(p, a, s);
     return T <= 8 ? launch_ffn<MOE_MXFP4, 1>(p, a, s) : launch_ffn<MOE_MXFP4, 2>(p, a, s);
+}
+
+}  // namespace moe
+
+extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx,
+                              const float* w, const int32_t* slot_of, float* y_part, void* y_bf16, int* status,
+                              void* stream) {
+    return expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, y_bf16, status, stream, 0);
 }
 
 extern "C" int moe_combine(const float* y_part, int T, int k, int H, void* y_bf16, void* stream) {

@@ -56,9 +56,11 @@ extern "C" int moe_decode_layer(moe_pool* p, int layer, const void* x_bf16, int 
 
 // All-resident decode of consecutive layers (post.smzdm.com/p/aomxznrn,
 // "FreeToken干的事": decode is scheduled on its own, bandwidth-bound path): per
-// layer the router, the lookup in its resident form and the FFN with the fused
-// combine, chained by programmatic stream serialisation with no host wait in
-// between, so a caller may capture the whole sequence in one CUDA graph.
+// layer the router and the FFN with the fused combine, the slot lookup folded
+// into the FFN's prologue (its resident form: slots from the key table, the
+// hits' LRU touch by CTA 0), chained by programmatic stream serialisation with
+// no host wait in between, so a caller may capture the whole sequence in one
+// CUDA graph.
 extern "C" int moe_decode_resident(moe_pool* p, int layer0, int n_layers, const void* x_bf16, int T,
                                    const void* const* wr_bf16, const float* const* bias, int renormalize,
                                    int32_t* idx, float* w, int32_t* slot_of, float* y_part, void* y_bf16,
@@ -67,7 +69,7 @@ extern "C" int moe_decode_resident(moe_pool* p, int layer0, int n_layers, const 
     const moe_config& c = p->cfg;
     if (n_layers <= 0 || layer0 < 0 || layer0 + n_layers > c.L) return fail(MOE_EBOUNDS, "layers outside the pool");
     if (T <= 0 || T > c.max_tokens) return fail(MOE_EINVAL, "T must be in [1, max_tokens]");
-    cudaStream_t s = (cudaStream_t)stream;
+    if (!slot_of) return fail(MOE_EINVAL, "null argument");
     const size_t xl = (size_t)T * c.H * 2;
     for (int i = 0; i < n_layers; i++) {
         if (!wr_bf16[i]) return fail(MOE_EINVAL, "null router weight");
@@ -76,8 +78,7 @@ extern "C" int moe_decode_resident(moe_pool* p, int layer0, int n_layers, const 
         int rc = moe_route(x, wr_bf16[i], bias ? bias[i] : nullptr, T, c.H, c.E, c.k, renormalize, idx, w, route_ws,
                            route_ws_bytes, stream);
         if (rc) return rc;
-        if ((rc = launch_lookup(p, layer0 + i, idx, T, c.k, slot_of, s, 1, status))) return rc;
-        if ((rc = moe_expert_ffn(p, layer0 + i, x, T, idx, w, slot_of, y_part, y, status, stream))) return rc;
+        if ((rc = expert_ffn(p, layer0 + i, x, T, idx, w, slot_of, y_part, y, status, stream, 1))) return rc;
     }
     return MOE_OK;
 }

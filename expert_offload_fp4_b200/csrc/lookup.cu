@@ -32,11 +32,6 @@ struct LookupArgs {
     int32_t* slot_of;
     LookupOut* out;
     int seq;
-    // resident mode: every expert must be resident already; no host record, no
-    // eviction, no ticket; a miss leaves the pool as it is (apart from the hits'
-    // clocks), gets slot -1 and sets MOE_STATUS_NOT_RESIDENT in *status
-    int resident;
-    int* status;
 };
 
 __device__ __forceinline__ bool key_less(unsigned long long ca, int sa, unsigned long long cb, int sb) {
@@ -73,11 +68,6 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(LookupArgs a) {
     }
     __syncthreads();
     if (s_bad) {
-        if (a.resident) {
-            if (tid == 0) atomicOr(a.status, MOE_STATUS_BAD_EXPERT);
-            for (int i = tid; i < a.n; i += blockDim.x) a.slot_of[i] = -1;
-            return;
-        }
         if (tid == 0) {
             a.out->n_uniq = 0;
             a.out->n_miss = 0;
@@ -134,14 +124,6 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(LookupArgs a) {
     }
     __syncthreads();
     const int nh = s_nh, nm = s_nm;
-    if (a.resident && nm > 0) {
-        if (tid == 0) {
-            *a.clock = G0 + nh;
-            atomicOr(a.status, MOE_STATUS_NOT_RESIDENT);
-        }
-        for (int i = tid; i < a.n; i += blockDim.x) a.slot_of[i] = uslot[umap[a.idx[i]]];   // -1 for a miss
-        return;
-    }
 
     // free slots, lowest index first: ranks by a block-wide scan over contiguous ranges
     const int per = (a.S + blockDim.x - 1) / blockDim.x;
@@ -240,21 +222,19 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(LookupArgs a) {
         *a.ticket = tk0 + nm;
     }
     __syncthreads();
-    if (!a.resident) {
-        for (int u = tid; u < nu; u += blockDim.x) {
-            a.out->uniq[u] = uniq[u];
-            a.out->is_hit[u] = 0;
-        }
+    for (int u = tid; u < nu; u += blockDim.x) {
+        a.out->uniq[u] = uniq[u];
+        a.out->is_hit[u] = 0;
     }
     __syncthreads();
-    if (tid == 0 && !a.resident) {
+    if (tid == 0) {
         // hits are the unique experts that are not in the miss list
         for (int u = 0; u < nu; u++) a.out->is_hit[u] = 1;
         for (int r = 0; r < nm; r++) a.out->is_hit[miss_u[r]] = 0;
     }
     for (int i = tid; i < a.n; i += blockDim.x) a.slot_of[i] = uslot[umap[a.idx[i]]];
     __syncthreads();
-    if (tid == 0 && !a.resident) {
+    if (tid == 0) {
         // the host polls seq in mapped memory: the record (and the miss list and
         // slot state above) must be visible system-wide before seq is
         a.out->n_uniq = nu;
@@ -275,20 +255,17 @@ int preload_lookup_kernels() {
 
 using namespace moe;
 
-namespace moe {
-
-// Enqueue the lookup kernel; resident != 0 is the all-resident form (status: its
-// device status word), which touches neither the host record nor its state.
-int launch_lookup(moe_pool* p, int layer, const int32_t* idx, int T, int k, int32_t* slot_of, cudaStream_t s,
-                  int resident, int* status) {
-    if (!p || !idx || !slot_of || (resident && !status)) return fail(MOE_EINVAL, "null argument");
+extern "C" int moe_slot_lookup_launch(moe_pool* p, int layer, const int32_t* idx, int T, int k,
+                                      int32_t* slot_of, void* stream) {
+    if (!p || !idx || !slot_of) return fail(MOE_EINVAL, "null argument");
     const moe_config& c = p->cfg;
     if (layer < 0 || layer >= c.L) return fail(MOE_EBOUNDS, "layer outside the pool");
     if (T <= 0 || k <= 0 || k > c.E || (long long)T * k > (1LL << 24)) return fail(MOE_EINVAL, "bad T/k");
     // the pool must hold every expert one call can touch, or a miss finds no victim
     const int cap = T * k < c.E ? T * k : c.E;
     if (cap > p->n_active) return fail(MOE_EINVAL, "slot pool smaller than the unique experts one call can touch");
-    if (!resident && p->lk_pending) return fail(MOE_ESTATE, "a launched lookup has not been collected");
+    if (p->lk_pending) return fail(MOE_ESTATE, "a launched lookup has not been collected");
+    cudaStream_t s = (cudaStream_t)stream;
     LookupArgs a;
     a.idx = idx;
     a.n = T * k;
@@ -303,9 +280,7 @@ int launch_lookup(moe_pool* p, int layer, const int32_t* idx, int T, int k, int3
     a.need = p->need;
     a.slot_of = slot_of;
     a.out = p->lk_d;
-    a.seq = resident ? 0 : ++p->lk_seq;
-    a.resident = resident;
-    a.status = status;
+    a.seq = ++p->lk_seq;
     const size_t smem = size_t(2) * ((p->n_active + 31) / 32) * sizeof(uint32_t);
     if (smem > 160 * 1024) return fail(MOE_EINVAL, "n_slots too large for the lookup kernel");
     if (!p->lk_attr_set) {
@@ -325,17 +300,9 @@ int launch_lookup(moe_pool* p, int layer, const int32_t* idx, int T, int k, int3
         lc.numAttrs = 1;
         MOE_CUDA_TRY(cudaLaunchKernelEx(&lc, lookup_kernel, a));
     }
-    if (resident) return MOE_OK;
     MOE_CUDA_TRY(cudaEventRecord(p->lk_event, s));
     p->lk_pending = 1;
     return MOE_OK;
-}
-
-}  // namespace moe
-
-extern "C" int moe_slot_lookup_launch(moe_pool* p, int layer, const int32_t* idx, int T, int k,
-                                      int32_t* slot_of, void* stream) {
-    return launch_lookup(p, layer, idx, T, k, slot_of, (cudaStream_t)stream, 0, nullptr);
 }
 
 extern "C" int moe_slot_lookup_result(moe_pool* p, moe_lookup_result* res) {

@@ -377,21 +377,23 @@ int moe_decode_layer(moe_pool* pool, int layer, const void* x_bf16, int T, const
 
 /* All-resident decode of layers layer0 .. layer0+n_layers-1 (post.smzdm.com/p/
  * aomxznrn, "FreeToken干的事": decode runs on its own bandwidth-bound path): per
- * layer moe_route, the slot lookup and moe_expert_ffn with the combine fused in,
- * on `stream`, with no host wait anywhere, so the call may be captured into a
- * CUDA graph and replayed.  Every expert the layers touch must already be
- * resident (for instance a pool with n_slots >= L * E after one pass of
- * moe_decode_layer): the lookup only refreshes the LRU clocks of its hits; it
- * never evicts, streams or writes the host record.  An expert that is not
- * resident leaves the pool untouched, sets MOE_STATUS_NOT_RESIDENT (and
- * MOE_STATUS_BAD_SLOT from the FFN) in *status, and that layer's output is not
- * valid.  x_bf16: [n_layers, T, H] (device); y_bf16: [n_layers, T, H];
- * wr_bf16, bias: host arrays of n_layers device pointers ([E, H] bf16 router
- * weights; [E] fp32 bias or NULL; bias itself may be NULL); idx, w, slot_of
- * ([T, k]), y_part ([T, k, H] fp32), route_ws and status as for
+ * layer moe_route and moe_expert_ffn with the combine fused in, the slot lookup
+ * folded into the FFN's prologue, on `stream`, with no host wait anywhere, so
+ * the call may be captured into a CUDA graph and replayed.  Every expert the
+ * layers touch must already be resident (for instance a pool with
+ * n_slots >= L * E after one pass of moe_decode_layer): each expert's slot comes
+ * from the pool's key table and the hits' LRU clocks are refreshed exactly as
+ * moe_slot_lookup refreshes them (ascending expert id); nothing is evicted,
+ * streamed or written to the lookup's host record; slot_of receives the slots.
+ * An expert that is not resident leaves the pool untouched apart from the hits'
+ * clocks, sets MOE_STATUS_NOT_RESIDENT and MOE_STATUS_BAD_SLOT in *status, and
+ * that layer's output is not valid.  x_bf16: [n_layers, T, H] (device); y_bf16:
+ * [n_layers, T, H]; wr_bf16, bias: host arrays of n_layers device pointers
+ * ([E, H] bf16 router weights; [E] fp32 bias or NULL; bias itself may be NULL);
+ * idx, w, slot_of ([T, k]), y_part ([T, k, H] fp32), route_ws and status as for
  * moe_decode_layer, reused by every layer in stream order.  No lookup may be
- * outstanding on the pool while the graph runs.  Errors: MOE_EINVAL,
- * MOE_EBOUNDS, and those of the three calls. */
+ * outstanding on the pool while it runs.  Errors: MOE_EINVAL, MOE_EBOUNDS, and
+ * those of moe_route and moe_expert_ffn. */
 int moe_decode_resident(moe_pool* pool, int layer0, int n_layers, const void* x_bf16, int T,
                         const void* const* wr_bf16, const float* const* bias, int renormalize,
                         int32_t* idx, float* w, int32_t* slot_of, float* y_part, void* y_bf16,
