@@ -70,7 +70,7 @@ def prefill_run(torch, m, w, T, experts, reps=5):
     cs = torch.cuda.Stream()
     m.stream_misses(pool, 0, res, cs)
     cs.synchronize()
-    y_part = torch.empty((T, 1, w.H), dtype=torch.float32, device="cuda")
+    y_part = torch.empty((T, w.k, w.H), dtype=torch.float32, device="cuda")
     y = torch.empty((T, w.H), dtype=torch.bfloat16, device="cuda")
     work = torch.zeros(m.prefill_workspace_bytes(pool, T), dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -305,8 +305,9 @@ def prefill_workspace_bytes(pool, T):
 
 
 def prefill_ffn(pool, layer, x, idx, w, slot_of, y, workspace, status, stream=None):
-    """y [T, H] fp32 (zeroed by the call) = the routed experts' FFN outputs summed
-    with their routing weights; round with combine(y.view(T, 1, H), y_bf16)."""
+    """y: y_part [T, k, H] fp32, every row written: the routed experts' FFN outputs
+    times their routing weights, one row per (token, rank); sum and round them in
+    rank order with combine(y, y_bf16)."""
     T = x.shape[0]
     L.check("moe_prefill_ffn", pool.lib.moe_prefill_ffn(
         pool.handle, int(layer), _p(x), T, _p(idx), _p(w), _p(slot_of), _p(y), _p(workspace),

@@ -277,7 +277,7 @@ struct GemmArgs {
     PrefillWs ws;
     const float* tscale;        // [L*E*3]
     const float* w;             // [T*k]
-    float* y;                   // [T*H] fp32, accumulated
+    float* y;                   // y_part [T, k, H] fp32: one row per (token, rank)
     int* status;
     int layer, E, k, H, I, NT;  // NT: N tiles per M tile
     long long b_gate_row, b_up_row, b_gsf_row, b_usf_row;  // row offsets inside a slot (GEMM1)
@@ -292,7 +292,7 @@ struct GemmArgs {
 // the A and B scale rows into scale-factor atoms; warp 1 issues the MMAs into one of two
 // TMEM accumulators, so warps 4-7 drain tile i while tile i+1 is multiplied.
 // MODE 1: gate/up with the SiLU * up + NVFP4 epilogue; MODE 2: down with the
-// routing-weight reduction into y.
+// routing weight, each row stored to its (token, rank) row of y_part.
 template <int MODE>
 __global__ void __launch_bounds__(kPThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_asf,
@@ -459,7 +459,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
                 if (tok >= 0) {
                     const int j = g.ws.perm_rank[row];
                     coef = g.w[tok * g.k + j] * ts[2];
-                    dst = g.y + (size_t)tok * g.H + n0;
+                    dst = g.y + ((size_t)tok * g.k + j) * g.H + n0;
                 }
 #pragma unroll
                 for (int c = 0; c < 4; c++) {
@@ -468,12 +468,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
                     if (tok >= 0) {
 #pragma unroll
                         for (int q = 0; q < 8; q++)
-                            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
-                                         ::"l"(dst + 32 * c + 4 * q), "f"(coef * __uint_as_float(r[4 * q])),
-                                           "f"(coef * __uint_as_float(r[4 * q + 1])),
-                                           "f"(coef * __uint_as_float(r[4 * q + 2])),
-                                           "f"(coef * __uint_as_float(r[4 * q + 3]))
-                                         : "memory");
+                            *reinterpret_cast<float4*>(dst + 32 * c + 4 * q) =
+                                make_float4(coef * __uint_as_float(r[4 * q]), coef * __uint_as_float(r[4 * q + 1]),
+                                            coef * __uint_as_float(r[4 * q + 2]), coef * __uint_as_float(r[4 * q + 3]));
                     }
                 }
             }
@@ -627,9 +624,6 @@ extern "C" int moe_prefill_ffn(moe_pool* p, int layer, const void* x_bf16, int T
     const int grid1 = std::min(PL.MT * g.NT, p->num_sms);
     grouped_gemm_kernel<1><<<grid1, kPThreads, smem, s>>>(ma1, msa1, mb1, msb1, g);
     MOE_CUDA_TRY(cudaGetLastError());
-    // y is zeroed only now, after GEMM1 has streamed its weights through L2, so that
-    // the down GEMM's reductions into it find it in L2
-    MOE_CUDA_TRY(cudaMemsetAsync(y, 0, size_t(T) * c.H * sizeof(float), s));
     // GEMM2 reads the down rows of the slot with its own pitch
     g.b_rows_per_slot = B.bytes / dr;
     g.b_sf_rows_per_slot = B.bytes / ds;

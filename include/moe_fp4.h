@@ -333,16 +333,17 @@ int moe_nvfp4_quantize(const void* x_bf16, int T, int H, uint8_t* codes, uint8_t
  * compute-bound and scheduled apart from decode).  Groups the (token, rank)
  * pairs by expert, quantises x to NVFP4 (as moe_nvfp4_quantize), runs the
  * gate/up GEMM on tcgen05 with a fused SiLU*up epilogue that re-quantises h to
- * NVFP4 (tensor scale 1), then the down GEMM with a fused routing-weight
- * combine: y[t, :] = sum_j w[t, j] * S_down * (W_down h)_t for expert idx[t, j]
- * read from slot slot_of[t, j] (all chosen experts resident); y is [T, H] fp32,
- * zeroed by the call and summed with fp32 vector reductions (the order of the
- * k terms is not fixed).
+ * NVFP4 (tensor scale 1), then the down GEMM, whose epilogue applies the
+ * routing weight and stores one row per (token, rank):
+ * y[t, j, :] = w[t, j] * S_down * (W_down h)_t for expert idx[t, j] read from
+ * slot slot_of[t, j] (all chosen experts resident); y is y_part [T, k, H] fp32,
+ * every row written by the call.
  * NVFP4 pools only; the expert block layout must divide into rows of H/2, H/16,
  * I/2 and I/16 bytes (MOE_EINVAL otherwise).  workspace: device memory of
  * moe_prefill_workspace_bytes(pool, T) bytes.  Device-side waits are bounded
- * and set bit 16 of *status (device int) on timeout.  moe_combine(y, T, 1, H, y_bf16)
- * rounds the result to bf16. */
+ * and set bit 16 of *status (device int) on timeout.  moe_combine(y, T, k, H,
+ * y_bf16) sums the k rows of each token in rank order in fp32 and rounds to
+ * bf16, as in decode, so the result does not depend on timing. */
 size_t moe_prefill_workspace_bytes(const moe_pool* pool, int T);
 int moe_prefill_ffn(moe_pool* pool, int layer, const void* x_bf16, int T, const int32_t* idx,
                     const float* w, const int32_t* slot_of, float* y, void* workspace,

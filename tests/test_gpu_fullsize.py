@@ -191,12 +191,12 @@ def test_prefill_35b_every_token(m):
     cs = torch.cuda.Stream()
     m.stream_misses(pool, 0, res, cs)
     cs.synchronize()
-    yacc = torch.full((T, w.H), float("nan"), dtype=torch.float32, device="cuda")
+    y_part = torch.full((T, w.k, w.H), float("nan"), dtype=torch.float32, device="cuda")
     work = torch.zeros(m.prefill_workspace_bytes(pool, T), dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    m.prefill_ffn(pool, 0, xd, idx, wt, slot_of, yacc, work, status)
+    m.prefill_ffn(pool, 0, xd, idx, wt, slot_of, y_part, work, status)
     y = torch.empty((T, w.H), dtype=torch.bfloat16, device="cuda")
-    m.combine(yacc.view(T, 1, w.H), y)
+    m.combine(y_part, y)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     idx_r, w_r, _ = oracle.route(x, wr, b, w.k, 1)
