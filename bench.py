@@ -445,6 +445,8 @@ def ffn_only(args, w, T):
         m._lib.load().moe_set_ffn_trace(None)
         tr = buf.cpu().numpy()
         n_cta = info["ctas"]
+        if args.trace_dump:
+            np.save(args.trace_dump, tr[:n_cta])
         tr = tr[:n_cta].astype(np.float64)
         t0 = tr[:, 0].min()
         names = {0: "start", 1: "staged", 2: "pdl", 3: "table", 4: "first_data", 5: "a_done",
@@ -690,6 +692,7 @@ def main():
     ap.add_argument("--workload", default="decode_35b", choices=["decode_35b", "decode_284b"],
                     help="--mode ffn: the layer shapes")
     ap.add_argument("--trace", action="store_true", help="--mode ffn: per-CTA phase stamps")
+    ap.add_argument("--trace-dump", default=None, help="--mode ffn --trace: also save the raw stamps (.npy)")
     ap.add_argument("--host-layers", type=int, default=8,
                     help="--mode offload: distinct host copies of the 40 layers (pinned RAM)")
     ap.add_argument("--no-overlap", action="store_true",

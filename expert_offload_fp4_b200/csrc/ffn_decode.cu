@@ -13,9 +13,9 @@
 // SM streams the same number of weight bytes whatever the number of groups.  B
 // waits (bounded) for A items of other CTAs; all CTAs are resident at once (one
 // per SM), and A items wait for nothing but their own copies and tickets, so the
-// waits always end.  The warp that lands the last group of a 16-row tile of H
-// (an atomic count per tile) sums y_part over the ranks in rank order and writes
-// the tile's bf16 output rows (K5).
+// waits always end.  Every B tile counts its 16-row tile of H (an atomic count
+// per tile); afterwards CTA c waits for the full counts of tiles c, c + grid, ...
+// and sums y_part over the ranks in rank order into their bf16 output rows (K5).
 //
 // Warp specialisation: warp 16 (the producer) streams the FP4 code rows and
 // block scales of each work stage with 1-D bulk copies (a tile of rows is one
@@ -468,6 +468,9 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
         if (bad && blockIdx.x == 0) atomicOr(a.status, bad);
     }
     __syncthreads();
+    // the producer's bulk (async proxy) reads of slots acquired above come after
+    // this fence; issued here, it overlaps the rest of the table
+    if (warp == kNC) fence_proxy_async_global();
     // leader (first entry of the same expert) and index among the expert's
     // entries, by one scan of the earlier entries (broadcast loads)
     if (tid < n && e_s[tid] >= 0) {
@@ -549,11 +552,10 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
         uint32_t round = 0;
         const uint8_t* blk = nullptr;
         // first use of a group's slot for gate/up (part 0) or down (part 1): a slot
-        // that showed that part when the table was built was acquired then (and
-        // the CTA barrier since orders it); for a pending one, wait (bounded) for
-        // the part's ticket and acquire it here.  Then the bulk (async proxy)
-        // reads are ordered after the acquire.
-        fence_proxy_async_global();
+        // that showed that part when the table was built was acquired then (the
+        // CTA barrier and the proxy fence after it order the bulk reads); for a
+        // pending one, wait (bounded) for the part's ticket, acquire it and fence
+        // here.
         if (trace && lane == 0) trace[9] = globaltimer();
         auto use_group = [&](int g, int part) {
             if (g == lastg && part == lastpart) return;
@@ -768,13 +770,12 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
                 for (int off = 8; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
                 if ((lane & 15) == 0 && o < 16 * M) atomicMax(pmax + pair, __float_as_uint(mx));
             }
-            // publish: the warp's h values and maxima are visible before the group's count grows
+            // publish: the warp's h values and maxima are visible before the group's
+            // count grows (the warp barrier orders the lanes' writes before lane 0's
+            // release add)
             cnt = __reduce_add_sync(0xffffffffu, cnt);
             __syncwarp();
-            if (lane == 0 && cnt) {
-                __threadfence();
-                atomicAdd(gcnt + g, (unsigned)cnt);
-            }
+            if (lane == 0 && cnt) red_release_add(gcnt + g, (unsigned)cnt);
             pst++;
         }
         named_sync(1, kConsThreads);      // x fragments are dead from here on
@@ -884,20 +885,23 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
                             G.wt[m] * (acc[n8][e] * hinv[m] * G.ts[2]);
                 }
             if (!a.y) continue;
-            // the row tile's part from this group is in y_part: count it; the warp
-            // that lands the last group sums the tile over the ranks in rank order
-            // and writes its bf16 rows (K5)
+            // the row tile's part from this group is in y_part: count it (release)
             __syncwarp();
-            unsigned prev = 0;
-            if (lane == 0) {
-                __threadfence();
-                prev = atomicAdd(rowcnt + rt, 1u);
-                if (prev == (unsigned)ng - 1u) __threadfence();
-            }
-            prev = __shfl_sync(0xffffffffu, prev, 0);
-            __syncwarp();                  // the lanes' loads below follow lane 0's fence
-            if (prev == (unsigned)ng - 1u) {
-                for (int v = lane; v < T * 16; v += 32) {
+            if (lane == 0) red_release_add(rowcnt + rt, 1u);
+        }
+        if (trace && tid == 0) trace[8] = globaltimer();
+
+        // ---- K5: CTA c sums the 16-row tiles rt = c, c + grid, ... of H over the
+        // ranks in rank order and writes their bf16 rows, once every group has
+        // counted them (bounded wait, acquire); the work is spread over the grid
+        if (a.y) {
+            for (int rt = blockIdx.x; rt < H / 16; rt += gridDim.x) {
+                if (tid == 0 && !wait_count(rowcnt + rt, (unsigned)ng, a.dep_ns, abort_flag)) {
+                    atomicOr(a.status, MOE_STATUS_DEP_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                named_sync(1, kConsThreads);
+                for (int v = tid; v < T * 16; v += kConsThreads) {
                     const int t = v >> 4, row = rt * 16 + (v & 15);
                     float sum = 0.0f;
                     for (int j = 0; j < a.k; j++) sum += __ldcg(a.y_part + ((size_t)t * a.k + j) * H + row);
@@ -905,7 +909,6 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
                 }
             }
         }
-        if (trace && tid == 0) trace[8] = globaltimer();
     }
 
     // ---- epilogue: the last CTA to finish clears the launch's counters and the
