@@ -223,7 +223,7 @@ def resident_run(torch, m, w, pool, T, x_dev, wr, bias, reps=10):
     wrs, bs = [wr] * L_, [bias] * L_
 
     def run(stream):
-        m.decode_resident(pool, 0, x_dev, wrs, bs, 1, idx, wt, slot_of, y_part, y, status, ws, stream=stream)
+        m.decode_resident(pool, 0, x_dev, wrs, bs, 1, idx, wt, slot_of, y_part, y, status, stream=stream)
 
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())

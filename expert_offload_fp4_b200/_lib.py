@@ -85,8 +85,7 @@ SIGNATURES = {
     "moe_combine": (i32, [vp, i32, i32, i32, vp, vp]),
     "moe_decode_layer": (i32, [vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,
                                C.POINTER(LookupResult), vp, vp, i32, vp, vp]),
-    "moe_decode_resident": (i32, [vp, i32, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t,
-                                  vp]),
+    "moe_decode_resident": (i32, [vp, i32, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp]),
     "qstar_split": (i32, [i32, f64, f64, C.POINTER(i32), C.POINTER(i32), C.POINTER(f64)]),
     "moe_bw_init": (i32, [C.POINTER(BwEstimate), f64, f64, f64]),
     "moe_bw_observe": (i32, [C.POINTER(BwEstimate), i32, f64, f64]),

@@ -209,11 +209,12 @@ def decode_layer(pool, layer, x, wr, bias, renormalize, idx, w, slot_of, y_part,
         _s(stream), _s(cs)))
 
 
-def decode_resident(pool, layer0, x, wr, bias, renormalize, idx, w, slot_of, y_part, y, status, ws, stream=None):
-    """moe_decode_resident: route, resident lookup and FFN (combine fused) of
-    x.shape[0] consecutive layers from layer0, with no host wait (capturable in a
-    CUDA graph).  x, y: [n_layers, T, H] bf16; wr: list of n_layers [E, H] bf16;
-    bias: list of n_layers [E] fp32 (entries may be None) or None."""
+def decode_resident(pool, layer0, x, wr, bias, renormalize, idx, w, slot_of, y_part, y, status, stream=None):
+    """moe_decode_resident: one FFN launch per layer with the router, the resident
+    lookup and the combine fused in, for x.shape[0] consecutive layers from
+    layer0, with no host wait (capturable in a CUDA graph).  x, y: [n_layers, T, H]
+    bf16; wr: list of n_layers [E, H] bf16; bias: list of n_layers [E] fp32
+    (entries may be None) or None."""
     n, T = x.shape[0], x.shape[1]
     if len(wr) != n or (bias is not None and len(bias) != n):
         raise ValueError("decode_resident: one router weight (and bias) per layer")
@@ -221,7 +222,7 @@ def decode_resident(pool, layer0, x, wr, bias, renormalize, idx, w, slot_of, y_p
     b_arr = None if bias is None else (C.c_void_p * n)(*[None if b is None else b.data_ptr() for b in bias])
     L.check("moe_decode_resident", pool.lib.moe_decode_resident(
         pool.handle, int(layer0), n, _p(x), T, wr_arr, b_arr, int(renormalize), _p(idx), _p(w), _p(slot_of),
-        _p(y_part), _p(y), _p(status), _p(ws), ws.numel(), _s(stream)))
+        _p(y_part), _p(y), _p(status), _s(stream)))
 
 
 def combine(y_part, y, stream=None):

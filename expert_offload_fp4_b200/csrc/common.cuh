@@ -65,10 +65,21 @@ int preload_gemm_kernels();
 int preload_prefill_kernels();
 int preload_pull_kernels();
 cudaError_t launch_pull(const uint8_t* src_d, uint8_t* dst, size_t bytes, int num_sms, cudaStream_t s);
+// The router fused into a resident decode FFN: router weights [E, H] bf16, bias
+// [E] or null, and the caller's idx / w, which the FFN writes.
+struct FfnRoute {
+    const void* wr;
+    const float* bias;
+    int renormalize;
+    int32_t* idx;
+    float* w;
+};
 // The decode FFN; resident != 0 takes the slots from the pool's key table and
-// applies the slot lookup's LRU touch itself (no lookup kernel before it).
+// applies the slot lookup's LRU touch itself (no lookup kernel before it); route
+// (resident only) routes the tokens inside the kernel (no router kernel either).
 int expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx, const float* w,
-               const int32_t* slot_of, float* y_part, void* y_bf16, int* status, void* stream, int resident);
+               const int32_t* slot_of, float* y_part, void* y_bf16, int* status, void* stream, int resident,
+               const FfnRoute* route);
 
 }  // namespace moe
 
@@ -105,10 +116,11 @@ struct moe_pool {
     int lk_attr_set;
     // decode FFN counters: [0, H/16) groups done per 16-row tile of H (the fused
     // combine), then per group the h values published, per (token, rank) the
-    // largest |h| (float bits), kMaxDecodePairs words each, then the abort flag
-    // and the count of finished CTAs
+    // largest |h| (float bits), kMaxDecodePairs words each, then the abort flag,
+    // the count of finished CTAs and the fused router's count of experts done
     unsigned int* ctr;
     float* hbuf;                  // decode FFN: [kMaxDecodePairs][I] h of each (token, rank)
+    float* rlogits;               // decode FFN's fused router: [kMaxDecodeT][E] logits
     // copy engine ready-flag write
     void* write_value32;          // cuStreamWriteValue32 entry point
     int ffn_grid[2][2];           // decode FFN CTAs per launch (0: not yet set up), per (format, token tiles)

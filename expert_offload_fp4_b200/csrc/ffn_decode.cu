@@ -36,6 +36,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "router_topk.cuh"
 
 namespace moe {
 
@@ -63,6 +64,8 @@ struct FfnArgs {
     const uint16_t* x;
     const int32_t* idx;
     const float* w;
+    int32_t* idx_out;          // fused router: the caller's idx and w, written by CTA 0
+    float* w_out;
     int32_t* slot_of;          // read; written by CTA 0 in resident mode
     float* y_part;
     uint16_t* y;               // bf16 output [T, H] (the fused combine), or null
@@ -80,6 +83,14 @@ struct FfnArgs {
     unsigned long long* slot_clock;
     unsigned long long* clock;
     int resident;
+    // fused router (resident mode only), or wr = null: idx and w come from the caller.
+    // Each of the first E consumer warps of the grid computes one expert's logits for
+    // every token in the router kernel's order; every CTA then selects the top-k of
+    // every token; CTA 0 writes idx and w for the caller.
+    const uint16_t* wr;        // [E][H] bf16
+    const float* rbias;        // [E] or null
+    int renorm;
+    float* rlogits;            // [T][E] fp32 scratch
     unsigned int* ctr;         // [H/16] row tiles, [kMaxDecodePairs] groups, [kMaxDecodePairs] pair maxima,
                                // abort flag, done count
     int T, k, H, I, E, S, layer;
@@ -359,6 +370,8 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     float* hinv = xinv + kMaxDecodeT;                                  // [16] per member
     unsigned* hmx = reinterpret_cast<unsigned*>(hinv + kMaxDecodeT);   // [16] per token (x staging)
     int* s_misc = reinterpret_cast<int*>(hmx + kMaxDecodeT);           // [8]
+    int32_t* ridx = reinterpret_cast<int32_t*>(s_misc + 8);            // [T*k] fused router's choices
+    float* rw = reinterpret_cast<float*>(ridx + kMaxDecodePairs);      // [T*k] and weights
     float* ts_row = reinterpret_cast<float*>(smem + a.o_ts);           // [E][3] this layer's tensor scales
     float* unitbuf = reinterpret_cast<float*>(smem + a.o_red);         // [unit][2][2 (gate, up)][ks][16][T]
     uint4* xf = reinterpret_cast<uint4*>(smem + a.o_frag);             // x fragments (A), N = T
@@ -373,6 +386,7 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     unsigned int* pmax = gcnt + kMaxDecodePairs;                       // [kMaxDecodePairs] max |h| bits per pair
     volatile unsigned int* abort_flag = pmax + kMaxDecodePairs;
     unsigned int* done_ctr = pmax + kMaxDecodePairs + 1;
+    unsigned int* route_ctr = pmax + kMaxDecodePairs + 2;              // experts whose logits are out
     const int bs = FMT == MOE_MXFP4 ? 32 : 16;
     const int nTA = I / 16, nTB = H / 16;                              // A items, B tiles per group
     const int nsegA = H / kSeg, nsegB = I / kSeg;
@@ -422,6 +436,16 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
             if (h == 0) xinv[t] = 1.0f / sc;
         }
     }
+    // fused router: this warp's expert's router row on its way to L2, and the raw
+    // bf16 x in the (still unused) stage ring after the top-k scratch
+    const int r_e = blockIdx.x * kNC + warp;
+    uint4* rx = reinterpret_cast<uint4*>(stages + (size_t)kNC * a.E * 5 + 15 - ((size_t)kNC * a.E * 5 + 15) % 16);
+    if (a.wr) {
+        if (warp < kNC && r_e < a.E)
+            for (int l = lane; l < H * 2 / 128; l += 32)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(a.wr + (size_t)r_e * H) + 128 * l));
+        for (int v = tid; v < T * H / 8; v += blockDim.x) rx[v] = __ldg(reinterpret_cast<const uint4*>(a.x) + v);
+    }
     __syncthreads();
     if (trace && tid == 0) trace[1] = globaltimer();
 
@@ -429,6 +453,71 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     pdl_wait();
     pdl_trigger();   // the next kernel may launch; it waits for this grid to finish
     if (trace && tid == 0) trace[2] = globaltimer();
+
+    // ---- fused router: fp32 logits in the router kernel's order (lane j sums, by
+    // fmaf in ascending h, the 8-element chunks c with c % 32 == j; then a xor
+    // butterfly 16 .. 1; the bias last), exchanged through global memory
+    if (a.wr) {
+        if (warp < kNC && r_e < a.E) {
+            float acc[kMaxDecodeT];
+#pragma unroll
+            for (int t = 0; t < kMaxDecodeT; t++) acc[t] = 0.0f;
+            const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + (size_t)r_e * H);
+            // chunks c = lane + 32 q in ascending q, four loads of W in flight at a time
+            for (int q0 = 0; q0 < H / 256; q0 += 4) {
+                uint4 wq[4];
+#pragma unroll
+                for (int i = 0; i < 4; i++) wq[i] = q0 + i < H / 256 ? __ldg(wrow + lane + 32 * (q0 + i)) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    if (q0 + i >= H / 256) break;
+                    const int c = lane + 32 * (q0 + i);
+                    const uint32_t wu[4] = {wq[i].x, wq[i].y, wq[i].z, wq[i].w};
+#pragma unroll
+                    for (int t = 0; t < kMaxDecodeT; t++) {
+                        if (t >= T) break;
+                        const uint4 xq = rx[(size_t)t * (H / 8) + c];
+                        const uint32_t xu[4] = {xq.x, xq.y, xq.z, xq.w};
+#pragma unroll
+                        for (int r = 0; r < 4; r++) {
+                            acc[t] = fmaf(__uint_as_float(xu[r] << 16), __uint_as_float(wu[r] << 16), acc[t]);
+                            acc[t] = fmaf(__uint_as_float(xu[r] & 0xFFFF0000u), __uint_as_float(wu[r] & 0xFFFF0000u),
+                                          acc[t]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < kMaxDecodeT; t++) {
+                if (t >= T) break;
+                float v = acc[t];
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0) a.rlogits[(size_t)t * a.E + r_e] = v + (a.rbias ? a.rbias[r_e] : 0.0f);
+            }
+            __syncwarp();
+            if (lane == 0) red_release_add(route_ctr, 1u);
+        }
+        if (tid == 0 && !wait_count(route_ctr, (unsigned)a.E, a.dep_ns, abort_flag)) {
+            atomicOr(a.status, MOE_STATUS_DEP_TIMEOUT);
+            *abort_flag = 1;
+        }
+        __syncthreads();
+        // top-k of token t by warp t (the stage ring is still unused: its first
+        // bytes hold the logits rows and the taken flags)
+        float* s_l = reinterpret_cast<float*>(stages) + (size_t)warp * a.E;
+        unsigned char* s_taken = stages + (size_t)kNC * a.E * 4 + (size_t)warp * a.E;
+        if (warp < T) {
+            for (int e = lane; e < a.E; e += 32) s_l[e] = __ldcg(a.rlogits + (size_t)warp * a.E + e);
+            __syncwarp();
+            router_topk_warp(s_l, s_taken, a.E, a.k, a.renorm, lane, ridx + warp * a.k, rw + warp * a.k);
+            if (blockIdx.x == 0 && lane < a.k) {
+                a.idx_out[warp * a.k + lane] = ridx[warp * a.k + lane];
+                a.w_out[warp * a.k + lane] = rw[warp * a.k + lane];
+            }
+        }
+        __syncthreads();
+    }
 
     // ---- prologue 2: the groups (unique experts) of the call, in ticket order.
     // The stage ring is still unused, so its first bytes hold the per-(token, rank)
@@ -446,7 +535,7 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     const int n = T * a.k;
     if (tid == 0) s_misc[0] = 0;
     if (tid < n) {
-        const int e = a.idx[tid];
+        const int e = a.wr ? ridx[tid] : a.idx[tid];
         int bad = 0;
         if (e < 0 || e >= a.E) bad |= MOE_STATUS_BAD_EXPERT;
         int sl = -1;
@@ -525,7 +614,7 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
         Group& G = groups[grank_s[lead_s[tid]]];
         G.tok[mi_s[tid]] = (uint8_t)(tid / a.k);
         G.rank[mi_s[tid]] = (uint8_t)(tid % a.k);
-        G.wt[mi_s[tid]] = a.w[tid];
+        G.wt[mi_s[tid]] = a.wr ? rw[tid] : a.w[tid];
     }
     __syncthreads();
     const int ng = s_misc[0];
@@ -925,6 +1014,7 @@ __global__ void __maxnreg__(kFfnMaxRegs) ffn_decode_kernel(const FfnArgs a) {
     if (s_misc[2]) {
         for (int i = tid; i < H / 16; i += blockDim.x) rowcnt[i] = 0u;
         for (int i = tid; i < 2 * kMaxDecodePairs; i += blockDim.x) gcnt[i] = 0u;   // counts and maxima
+        if (tid == 0) *route_ctr = 0u;
         __syncthreads();
         if (tid == 0) {
             *abort_flag = 0u;
@@ -990,7 +1080,7 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
 static size_t up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
 // Shared-memory layout, ring and B stage shape of a launch with T tokens.
-static int plan_ffn(const moe_pool* p, int T, FfnArgs& a, size_t& smem) {
+static int plan_ffn(const moe_pool* p, int T, FfnArgs& a, size_t& smem, bool fused_router) {
     const moe_config& c = p->cfg;
     const int bs = p->bs;
     const size_t SA = c.H / bs, SB = c.I / bs;
@@ -1009,7 +1099,7 @@ static int plan_ffn(const moe_pool* p, int T, FfnArgs& a, size_t& smem) {
     a.o_groups = (int)o;
     o += sizeof(Group) * std::min(kMaxDecodePairs, c.max_tokens * c.k);
     a.o_misc = (int)up(o, 16);
-    o = a.o_misc + 3 * kMaxDecodeT * sizeof(float) + 8 * sizeof(int);
+    o = a.o_misc + 3 * kMaxDecodeT * sizeof(float) + 8 * sizeof(int) + 2 * kMaxDecodePairs * 4;
     a.o_ts = (int)up(o, 16);
     o = a.o_ts + (size_t)c.E * 3 * sizeof(float);
     a.o_red = (int)up(o, 16);
@@ -1018,7 +1108,9 @@ static int plan_ffn(const moe_pool* p, int T, FfnArgs& a, size_t& smem) {
     o = a.o_frag + std::max((size_t)T * c.H * 2, (size_t)2 * T * c.I * 2);
     a.o_stage = (int)up(o, 128);
     // the prologue keeps its per-(token, rank) table (9 ints + a u64 each) in the ring
-    const size_t need_ring = std::max((size_t)2 * a.stage_bytes, (size_t)11 * 4 * kMaxDecodePairs);
+    // (and the fused router its logits rows and flags, kNC * E * 5 bytes, then x)
+    const size_t need_ring = std::max({(size_t)2 * a.stage_bytes, (size_t)11 * 4 * kMaxDecodePairs,
+                                       fused_router ? up((size_t)kNC * c.E * 5, 16) + (size_t)T * c.H * 2 : 0});
     if (a.o_stage + need_ring > budget)
         return fail(MOE_EINVAL, "decode FFN: T * H too large for shared memory (lower max_tokens)");
     // a power of two (at most 8), so that 2, 4 or 8 consumer units can share the ring
@@ -1052,7 +1144,7 @@ static int launch_ffn(moe_pool* p, FfnArgs& a, cudaStream_t s) {
     int grid = 0;
     int rc = ffn_grid<FMT, NT>(p, grid);
     if (rc) return rc;
-    rc = plan_ffn(p, a.T, a, smem);
+    rc = plan_ffn(p, a.T, a, smem, a.wr != nullptr);
     if (rc) return rc;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(grid);
@@ -1107,7 +1199,7 @@ extern "C" int moe_ffn_launch_info(moe_pool* p, int T, int* ctas, int* nstage, i
     else
         rc = T <= 8 ? ffn_grid<MOE_MXFP4, 1>(p, grid) : ffn_grid<MOE_MXFP4, 2>(p, grid);
     if (rc) return rc;
-    rc = plan_ffn(p, T, a, smem);
+    rc = plan_ffn(p, T, a, smem, false);
     if (rc) return rc;
     *ctas = grid;
     *nstage = a.nstage;
@@ -1127,7 +1219,10 @@ extern "C" int moe_set_wait_limits(double ready_ms, double dep_ms, double pipe_m
 namespace moe {
 
 int expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx, const float* w,
-               const int32_t* slot_of, float* y_part, void* y_bf16, int* status, void* stream, int resident) {
+               const int32_t* slot_of, float* y_part, void* y_bf16, int* status, void* stream, int resident,
+               const FfnRoute* route) {
+    if (route && !resident) return fail(MOE_EINVAL, "decode FFN: the fused router needs resident mode");
+    if (route && (!route->wr || !route->idx || !route->w)) return fail(MOE_EINVAL, "null argument");
     if (!p || !x_bf16 || !idx || !w || !slot_of || !y_part || !status) return fail(MOE_EINVAL, "null argument");
     const moe_config& c = p->cfg;
     if (layer < 0 || layer >= c.L) return fail(MOE_EBOUNDS, "layer outside the pool");
@@ -1151,6 +1246,14 @@ int expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t*
     a.ctr = p->ctr;
     a.hbuf = p->hbuf;
     a.resident = resident;
+    if (route) {
+        a.wr = (const uint16_t*)route->wr;
+        a.rbias = route->bias;
+        a.renorm = route->renormalize;
+        a.rlogits = p->rlogits;
+        a.idx_out = route->idx;
+        a.w_out = route->w;
+    }
     a.key_slot = p->key_slot;
     a.slot_clock = p->slot_clock;
     a.clock = p->clock;
@@ -1175,7 +1278,7 @@ int expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t*
 extern "C" int moe_expert_ffn(moe_pool* p, int layer, const void* x_bf16, int T, const int32_t* idx,
                               const float* w, const int32_t* slot_of, float* y_part, void* y_bf16, int* status,
                               void* stream) {
-    return expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, y_bf16, status, stream, 0);
+    return expert_ffn(p, layer, x_bf16, T, idx, w, slot_of, y_part, y_bf16, status, stream, 0, nullptr);
 }
 
 extern "C" int moe_combine(const float* y_part, int T, int k, int H, void* y_bf16, void* stream) {

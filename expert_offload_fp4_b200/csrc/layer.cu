@@ -55,30 +55,29 @@ extern "C" int moe_decode_layer(moe_pool* p, int layer, const void* x_bf16, int 
 }
 
 // All-resident decode of consecutive layers (post.smzdm.com/p/aomxznrn,
-// "FreeToken干的事": decode is scheduled on its own, bandwidth-bound path): per
-// layer the router and the FFN with the fused combine, the slot lookup folded
-// into the FFN's prologue (its resident form: slots from the key table, the
-// hits' LRU touch by CTA 0), chained by programmatic stream serialisation with
-// no host wait in between, so a caller may capture the whole sequence in one
-// CUDA graph.
+// "FreeToken干的事": decode is scheduled on its own, bandwidth-bound path): one
+// FFN launch per layer with the router, the slot lookup (its resident form: slots
+// from the key table, the hits' LRU touch by CTA 0) and the combine fused in,
+// chained by programmatic stream serialisation with no host wait in between, so
+// a caller may capture the whole sequence in one CUDA graph.
 extern "C" int moe_decode_resident(moe_pool* p, int layer0, int n_layers, const void* x_bf16, int T,
                                    const void* const* wr_bf16, const float* const* bias, int renormalize,
                                    int32_t* idx, float* w, int32_t* slot_of, float* y_part, void* y_bf16,
-                                   int* status, void* route_ws, size_t route_ws_bytes, void* stream) {
+                                   int* status, void* stream) {
     if (!p || !x_bf16 || !wr_bf16 || !y_bf16 || !status) return fail(MOE_EINVAL, "null argument");
     const moe_config& c = p->cfg;
     if (n_layers <= 0 || layer0 < 0 || layer0 + n_layers > c.L) return fail(MOE_EBOUNDS, "layers outside the pool");
     if (T <= 0 || T > c.max_tokens) return fail(MOE_EINVAL, "T must be in [1, max_tokens]");
-    if (!slot_of) return fail(MOE_EINVAL, "null argument");
+    if (!slot_of || !idx || !w || !y_part) return fail(MOE_EINVAL, "null argument");
+    if (renormalize != 0 && renormalize != 1) return fail(MOE_EINVAL, "renormalize must be 0 or 1");
     const size_t xl = (size_t)T * c.H * 2;
     for (int i = 0; i < n_layers; i++) {
         if (!wr_bf16[i]) return fail(MOE_EINVAL, "null router weight");
         const uint8_t* x = (const uint8_t*)x_bf16 + i * xl;
         uint8_t* y = (uint8_t*)y_bf16 + i * xl;
-        int rc = moe_route(x, wr_bf16[i], bias ? bias[i] : nullptr, T, c.H, c.E, c.k, renormalize, idx, w, route_ws,
-                           route_ws_bytes, stream);
+        const FfnRoute route{wr_bf16[i], bias ? bias[i] : nullptr, renormalize, idx, w};
+        const int rc = expert_ffn(p, layer0 + i, x, T, idx, w, slot_of, y_part, y, status, stream, 1, &route);
         if (rc) return rc;
-        if ((rc = expert_ffn(p, layer0 + i, x, T, idx, w, slot_of, y_part, y, status, stream, 1))) return rc;
     }
     return MOE_OK;
 }

@@ -88,6 +88,7 @@ extern "C" int moe_pool_destroy(moe_pool* p) {
     cudaFree(p->tscale);
     cudaFree(p->ctr);
     cudaFree(p->hbuf);
+    cudaFree(p->rlogits);
     if (p->host) cudaFreeHost(p->host);
     if (p->lk_h) cudaFreeHost(p->lk_h);
     if (p->lk_event) cudaEventDestroy(p->lk_event);
@@ -138,6 +139,7 @@ extern "C" int moe_pool_create(const moe_config* cfg, moe_pool** out) {
     ALLOC(p->tscale, LE * 3 * sizeof(float));
     ALLOC(p->ctr, ((size_t)cfg->H / 16 + 2 * kMaxDecodePairs + 8) * sizeof(unsigned int));
     ALLOC(p->hbuf, (size_t)kMaxDecodePairs * cfg->I * sizeof(float));
+    ALLOC(p->rlogits, (size_t)kMaxDecodeT * cfg->E * sizeof(float));
 #undef ALLOC
     cudaMemset(p->slot_key, 0xFF, S * sizeof(int32_t));
     cudaMemset(p->slot_clock, 0, S * sizeof(unsigned long long));

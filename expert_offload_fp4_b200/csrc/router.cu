@@ -11,6 +11,7 @@
 // CTA) selects the top-k of each token with one warp (descending logit, ties to
 // the lower index) and writes the softmax weights.
 #include "common.cuh"
+#include "router_topk.cuh"
 
 namespace moe {
 
@@ -125,53 +126,10 @@ router_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr,
     __shared__ unsigned char s_taken[kRouterWarps][kMaxE];
     for (int t = warp; t < nt; t += kRouterWarps) {
         const float* row = logits + size_t(t0 + t) * E;
-        for (int e = lane; e < E; e += 32) {
-            s_l[warp][e] = __ldcg(row + e);
-            s_taken[warp][e] = 0;
-        }
+        for (int e = lane; e < E; e += 32) s_l[warp][e] = __ldcg(row + e);
         __syncwarp();
-        float my_l = 0.0f;
-        int my_e = -1;
-        for (int j = 0; j < k; j++) {
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-            for (int e = lane; e < E; e += 32) {
-                const float v = s_l[warp][e];
-                if (!s_taken[warp][e] && (v > bv || (v == bv && e < be) || be == 0x7fffffff)) {
-                    bv = v;
-                    be = e;
-                }
-            }
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-                    bv = ov;
-                    be = oe;
-                }
-            }
-            if (lane == 0) s_taken[warp][be] = 1;
-            if (lane == j) {
-                my_l = bv;
-                my_e = be;
-            }
-            __syncwarp();
-        }
-        const float lmax = __shfl_sync(0xffffffffu, my_l, 0);
-        float den = 0.0f;
-        if (renorm) {
-            den = lane < k ? expf(my_l - lmax) : 0.0f;
-        } else {
-            for (int e = lane; e < E; e += 32) den += expf(s_l[warp][e] - lmax);
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-        if (lane < k) {
-            idx[size_t(t0 + t) * k + lane] = my_e;
-            wout[size_t(t0 + t) * k + lane] = expf(my_l - lmax) / den;
-        }
-        __syncwarp();
+        router_topk_warp(s_l[warp], s_taken[warp], E, k, renorm, lane, idx + size_t(t0 + t) * k,
+                         wout + size_t(t0 + t) * k);
     }
     if (threadIdx.x == 0) tile_cnt[blockIdx.y] = 0;
 }

@@ -377,10 +377,11 @@ int moe_decode_layer(moe_pool* pool, int layer, const void* x_bf16, int T, const
                      void* copy_end, int overlap, void* stream, void* copy_stream);
 
 /* All-resident decode of layers layer0 .. layer0+n_layers-1 (post.smzdm.com/p/
- * aomxznrn, "FreeToken干的事": decode runs on its own bandwidth-bound path): per
- * layer moe_route and moe_expert_ffn with the combine fused in, the slot lookup
- * folded into the FFN's prologue, on `stream`, with no host wait anywhere, so
- * the call may be captured into a CUDA graph and replayed.  Every expert the
+ * aomxznrn, "FreeToken干的事": decode runs on its own bandwidth-bound path): one
+ * decode FFN launch per layer with the router (the same logits, choices and
+ * weights as moe_route, bit for bit), the slot lookup and the combine fused in,
+ * on `stream`, with no host wait anywhere, so the call may be captured into a
+ * CUDA graph and replayed.  Every expert the
  * layers touch must already be resident (for instance a pool with
  * n_slots >= L * E after one pass of moe_decode_layer): each expert's slot comes
  * from the pool's key table and the hits' LRU clocks are refreshed exactly as
@@ -391,14 +392,15 @@ int moe_decode_layer(moe_pool* pool, int layer, const void* x_bf16, int T, const
  * that layer's output is not valid.  x_bf16: [n_layers, T, H] (device); y_bf16:
  * [n_layers, T, H]; wr_bf16, bias: host arrays of n_layers device pointers
  * ([E, H] bf16 router weights; [E] fp32 bias or NULL; bias itself may be NULL);
- * idx, w, slot_of ([T, k]), y_part ([T, k, H] fp32), route_ws and status as for
- * moe_decode_layer, reused by every layer in stream order.  No lookup may be
- * outstanding on the pool while it runs.  Errors: MOE_EINVAL, MOE_EBOUNDS, and
- * those of moe_route and moe_expert_ffn. */
+ * idx, w, slot_of ([T, k], written: the last layer's choices, weights and
+ * slots), y_part ([T, k, H] fp32) and status as for moe_decode_layer, reused by
+ * every layer in stream order.  No lookup may be outstanding on the pool while
+ * it runs, and calls on one pool must not run concurrently.  Errors:
+ * MOE_EINVAL, MOE_EBOUNDS, and those of moe_expert_ffn. */
 int moe_decode_resident(moe_pool* pool, int layer0, int n_layers, const void* x_bf16, int T,
                         const void* const* wr_bf16, const float* const* bias, int renormalize,
                         int32_t* idx, float* w, int32_t* slot_of, float* y_part, void* y_bf16,
-                        int* status, void* route_ws, size_t route_ws_bytes, void* stream);
+                        int* status, void* stream);
 
 /* q* split (post.smzdm.com/p/a825qpgl section 二: q* = m*B_p/B_h; "跑不快大模型，
  * 先别急着怪显卡" section 二: pull : compute = pcie_bw : (cpu_bw - pcie_bw)).

@@ -62,7 +62,7 @@ class Buffers:
 
     def run(self, m, pool, x, wr, bias, stream=None):
         m.decode_resident(pool, 0, x, wr, bias, 1, self.idx, self.w, self.slot_of, self.y_part, self.y,
-                          self.status, self.ws, stream=stream)
+                          self.status, stream=stream)
 
 
 CASES = [("35b_t1", W.DECODE_35B, 1), ("35b_t8", W.DECODE_35B, 8), ("tiny_t4", W.TINY, 4)]
@@ -95,7 +95,10 @@ def test_resident_equals_per_layer_and_oracle(m, name, w, T):
     b.run(m, pool_b, x, wr, bias)
     torch.cuda.synchronize()
     assert int(b.status.item()) == 0
-    assert np.array_equal(b.slot_of.cpu().numpy(), lo.slot_of.cpu().numpy())   # the last layer's slots
+    # the last layer's choices, weights and slots
+    assert np.array_equal(b.idx.cpu().numpy(), lo.idx.cpu().numpy())
+    assert np.array_equal(b.w.cpu().numpy().view(np.uint32), lo.w.cpu().numpy().view(np.uint32))
+    assert np.array_equal(b.slot_of.cpu().numpy(), lo.slot_of.cpu().numpy())
     for layer in range(L):
         got = b.y[layer].view(torch.int16).cpu().numpy()
         assert np.array_equal(got, y_ref[layer].view(torch.int16).cpu().numpy()), layer
