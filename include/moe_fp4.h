@@ -301,11 +301,12 @@ int moe_ffn_launch_info(moe_pool* pool, int T, int* ctas, int* nstage, int* stag
  * in ns: [0] start, [1] activations staged, [2] the preceding kernel (the slot
  * lookup) complete, [3] group table built, [4] first weights landed, [5] the
  * CTA's gate/up tiles done, [6] h of its first down tile's expert complete,
- * [7] that h in shared memory, [8] the CTA's down tiles done, [10] end,
- * [11] the producer's last copy issued, [16 + s] the CTA's stage s landed
- * (consumer side, s < 8), [24 + s] the producer's copies of stage s issued
- * (s < 8); and counts: [12] gate/up tiles of the CTA, [13] its down tiles,
- * [14] the K split of its gate/up units.
+ * [7] that h in shared memory, [8] the CTA's down tiles done, [9] the producer
+ * about to issue its first copy, [10] end, [11] the producer's last copy
+ * issued, [16 + s] the CTA's stage s landed (consumer side, s < 8), [24 + s] the
+ * producer's copies of stage s issued (s < 8); and counts: [12] gate/up tiles
+ * of the CTA, [13] its down tiles, [14] the K split of its gate/up units, [15]
+ * the K split of its down groups.
  * Unwritten entries keep their old value.  NULL turns tracing off. */
 int moe_set_ffn_trace(void* buf);
 
