@@ -37,6 +37,26 @@ def test_every_declared_symbol_is_exported(lib):
         assert n in lib.SIGNATURES, f"{n} has no binding signature"
 
 
+def declared_arities():
+    """{name: number of parameters} of every function the header declares."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(([^;]*?)\)\s*;", src,
+                         flags=re.M | re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every ctypes signature has as many arguments as the header's declaration."""
+    ar = declared_arities()
+    assert set(ar) == set(declared_functions())
+    for name, n in ar.items():
+        assert len(lib.SIGNATURES[name][1]) == n, (name, n, len(lib.SIGNATURES[name][1]))
+
+
 def test_qstar_split_through_the_abi_matches_table(lib):
     import expert_offload_fp4_b200 as m
     for _, bp, bh, pct in read_golden("qstar_table.txt"):
