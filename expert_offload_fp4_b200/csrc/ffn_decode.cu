@@ -49,6 +49,8 @@ constexpr int kConsThreads = kNC * 32;
 // must fit beside them: 5 * 32 * 96 + 32 * 32 <= 16384.
 constexpr int kFfnMaxRegs = 96;
 constexpr int kSeg = 128;                    // K elements per segment (64 code bytes)
+// SMs left free for the SM copy kernel (MOE_COPY_SM), which a waiting FFN depends on
+constexpr int kCopySMs = 16;
 
 struct Group {
     int expert, slot, M;
@@ -1135,6 +1137,8 @@ static int ffn_grid(moe_pool* p, int& grid) {
         p->ffn_grid[fi][ni] = p->num_sms;   // one per SM: more would only wait
     }
     grid = p->ffn_grid[fi][ni];
+    // the SM copy kernel streams misses the FFN waits for: leave it SMs of its own
+    if (p->copy_mode == MOE_COPY_SM) grid = std::max(1, grid - kCopySMs);
     return MOE_OK;
 }
 

@@ -246,9 +246,8 @@ int moe_stream_misses(moe_pool* pool, int layer, const moe_miss* miss_h, int n_m
 
 /* Select how moe_stream_misses copies (MOE_COPY_SM or MOE_COPY_DMA) for later
  * calls on this pool.  Both write the same bytes and publish the same ready
- * tickets.  The copy kernel of MOE_COPY_SM runs beside a waiting decode FFN
- * (one 128-thread CTA per SM fits next to an FFN CTA: the FFN caps its
- * registers and shared memory for that).  Errors: MOE_EINVAL. */
+ * tickets.  In MOE_COPY_SM mode the decode FFN runs on 16 SMs fewer, which the
+ * copy kernel it waits for uses.  Errors: MOE_EINVAL. */
 int moe_pool_set_copy_mode(moe_pool* pool, int mode);
 
 /* Decode expert FFN (post.smzdm.com/p/aomxznrn, "FreeToken干的事": decode is
