@@ -21,6 +21,12 @@ def test_expert_bytes_of_the_35b_layer():
     assert bench.expert_bytes_alg(W.DECODE_35B) == 3 * (2048 * 768 // 2 + 2048 * 768 // 16)
 
 
+def test_ffn_launch_bytes_include_the_fused_combine():
+    # 8 experts x 2,654,208 B of weights + x (T*H bf16) + y_part (T*k*H fp32) + y (T*H bf16)
+    assert bench.ffn_alg_bytes(W.DECODE_35B, 1, 8) == 8 * 2654208 + 4096 + 65536 + 4096 == 21307392
+    assert bench.ffn_alg_bytes(W.DECODE_35B, 8, 20) == 20 * 2654208 + 8 * 2048 * (2 + 8 * 4 + 2)
+
+
 def test_overlap_efficiency_definition():
     assert bench.overlap_efficiency(10.0, 10.0, 4.0) == 1.0        # fully hidden
     assert bench.overlap_efficiency(14.0, 10.0, 4.0) == 0.0        # serialised
